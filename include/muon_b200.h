@@ -1,0 +1,178 @@
+/*
+ * muon_b200.h -- C ABI of the Muon optimizer step for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (sources are the pages the method is described on):
+ *
+ *  - Muon step, "Muon优化器" (Muon optimizer, linsight.cn/f25d614e.html), section
+ *    "Muon 算法伪代码与 PyTorch 实现": for every 2-D weight W (rows = d_out, cols = d_in)
+ *      M <- beta*M + G                       (heavy-ball momentum, fp32 buffer)
+ *      U <- nesterov ? beta*M + G : M
+ *      X0 <- bf16(U), X <- X0 / (||X0||_F + eps)            ("zeropower_via_newtonschulz")
+ *      T times: A = X X^T, B = b A + c A A, X = a X + B X   (X^T X form when rows > cols)
+ *      W <- (1 - lr*wd) W - lr * scale(rows, cols) * X      (decoupled weight decay)
+ *    with per-iteration (a, b, c): the fixed schedule (3.4445, -4.7750, 2.0315) x 5 of the
+ *    section "Newton-Schulz 迭代", or the hybrid 8 fast + 2 stabilising iterations of
+ *    prism.simon-ai.net/article/8795 (DeepSeek V4 section); the scale is one of the four
+ *    of the section "缩放因子" (Moonlight 0.2*sqrt(max), KellerJordan, muP, naive).
+ *  - Stiefel variant, "Muon 在 Stiefel 流形上的精确闭式更新" (mlqm.cn/news/1339166):
+ *      V = G - W sym(W^T G)                                  (§1.3 / §3.2 tangent projection)
+ *      W <- (I + c A)^-1 (I - c A) W, A = V W^T - W V^T, c = lr/2   (§3.2 Cayley)
+ *    evaluated in the rank-2k Woodbury form of §6.2 (a 2k x 2k solve plus n x k GEMMs).
+ *
+ * Conventions shared by every entry point:
+ *  - All matrices are dense row-major.  Matrix pointers are DEVICE pointers; descriptor
+ *    arrays, schedules and coefficient tables are HOST pointers read during the call only.
+ *  - The caller owns every buffer, including the workspace; the library never allocates
+ *    device memory.  The workspace holds the library's tables between calls: a call with
+ *    the same arguments and workspace as the previous call on that workspace reuses them
+ *    (it then issues kernel launches only).  Do not write to a workspace between calls.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every entry point is
+ *    asynchronous on `stream` and never synchronises it, except
+ *    muon_workspace_device_status(), which does.
+ *  - Host-side argument checks run before any launch; on error nothing is launched and
+ *    buffers are untouched.  Launch failures return MUON_ERR_CUDA.  Device-side
+ *    conditions (a non-finite Frobenius norm, a kernel wait that ran out of time) are
+ *    recorded in the workspace and read back by muon_workspace_device_status().
+ *  - bf16 matrices handled on the tensor-core path need rows % 8 == 0, cols % 8 == 0 and
+ *    16-byte aligned pointers (TMA and 128-bit accesses); fp32 mode has no shape limit
+ *    beyond 16-byte aligned pointers.  Workspaces must be 256-byte aligned (they hold TMA
+ *    tensor maps); torch and cudaMalloc allocations are.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MUON_OK = 0,
+    MUON_ERR_INVALID_ARG = 1,          /* null pointer, count <= 0, bad enum, bad schedule   */
+    MUON_ERR_UNSUPPORTED_SHAPE = 2,    /* rows/cols not a multiple of 8 on the bf16 path;
+                                          n < k for Stiefel; a dimension above the limits */
+    MUON_ERR_ALIGNMENT = 3,            /* a device pointer not 16-byte aligned            */
+    MUON_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the *_workspace_size() minimum    */
+    MUON_ERR_CUDA = 5,                 /* a CUDA runtime/driver call failed               */
+    MUON_ERR_NONFINITE = 6,            /* device status: a NaN/Inf Frobenius norm          */
+    MUON_ERR_DEVICE_TIMEOUT = 7        /* device status: a kernel wait gave up (bounded)  */
+} muon_status;
+
+typedef enum { MUON_BF16 = 0, MUON_F32 = 1 } muon_dtype;
+
+/* Update scale for W in R^{d_out x d_in} (Muon optimizer page, section "缩放因子"). */
+typedef enum {
+    MUON_SCALE_MOONLIGHT = 0,   /* 0.2 * sqrt(max(d_out, d_in))  */
+    MUON_SCALE_KJ = 1,          /* sqrt(max(1, d_out / d_in))    */
+    MUON_SCALE_MUP = 2,         /* sqrt(d_out / d_in)            */
+    MUON_SCALE_NAIVE = 3        /* 1                             */
+} muon_scale_mode;
+
+#define MUON_MAX_NS_ITERS 32
+
+/* Newton-Schulz schedule.  Iteration t (0-based) uses a = coeffs[3t], b = coeffs[3t+1],
+ * c = coeffs[3t+2].  The first n_split_iters iterations run in split-bf16 (every operand
+ * and intermediate kept as a bf16 hi + lo pair, three tensor-core products per GEMM:
+ * hi*hi + hi*lo + lo*hi); later ones in plain bf16.  fp32_mode = 1 skips the bf16 cast and
+ * runs every product in fp32 FMA arithmetic (no TF32).  eps is added to the Frobenius norm
+ * (the page uses 1e-7). */
+typedef struct {
+    int n_iters;              /* 0 .. MUON_MAX_NS_ITERS (0: X = X0 / (||X0|| + eps)) */
+    const float* coeffs;      /* host, 3 * n_iters floats                                */
+    int n_split_iters;        /* 0 .. n_iters; ignored when fp32_mode                     */
+    int fp32_mode;            /* 0 or 1                                                  */
+    float eps;                /* > 0                                                     */
+} muon_ns_schedule;
+
+/* One Muon matrix.  W is updated in place (w_dtype), M (fp32) is updated in place, G is
+ * read (g_dtype).  O_out, if not NULL, receives the orthogonalised update X of Newton-
+ * Schulz (before the shape scale) as rows x cols bf16 (fp32 in fp32 mode). */
+typedef struct {
+    void* W;
+    const void* G;
+    float* M;
+    void* O_out;
+    int rows;
+    int cols;
+    int w_dtype;              /* muon_dtype */
+    int g_dtype;              /* muon_dtype */
+} muon_matrix_desc;
+
+typedef struct {
+    float lr;
+    float beta;               /* momentum coefficient (page default 0.95)                 */
+    float weight_decay;       /* decoupled: W <- (1 - lr*wd) W before the step             */
+    int nesterov;             /* 0: NS input is M; 1: beta*M + G                          */
+    int scale_mode;           /* muon_scale_mode                                          */
+    muon_ns_schedule ns;
+} muon_hyper;
+
+/* Bytes of workspace muon_step_batched needs for this set (0 if the arguments are
+ * invalid).  The set is processed in one pass when ws_bytes is at least this size; a
+ * smaller workspace of at least muon_step_workspace_min() is processed in groups. */
+MUON_API size_t muon_step_workspace_size(const muon_matrix_desc* descs, int count, const muon_hyper* hp);
+MUON_API size_t muon_step_workspace_min(const muon_matrix_desc* descs, int count, const muon_hyper* hp);
+
+/* One full Muon step (momentum, bf16 cast, Frobenius pre-scale, Newton-Schulz, shape
+ * scale, decoupled weight decay, update) for `count` matrices of any shapes.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, ALIGNMENT, WORKSPACE_TOO_SMALL, CUDA. */
+MUON_API muon_status muon_step_batched(const muon_matrix_desc* descs, int count, const muon_hyper* hp,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* Newton-Schulz orthogonalisation (Muon optimizer page, zeropower_via_newtonschulz) of a
+ * contiguous batch of rows x cols matrices: X_out[i] ~ msign(X_in[i]).  X_in is read as
+ * in_dtype; in bf16 mode an fp32 input is first rounded to bf16 (the page's cast).
+ * X_out is written as out_dtype.  X_in and X_out may not overlap. */
+MUON_API size_t ns_workspace_size(int batch, int rows, int cols, const muon_ns_schedule* sch);
+MUON_API muon_status ns_orthogonalize(const void* X_in, int in_dtype, void* X_out, int out_dtype,
+                             int batch, int rows, int cols, const muon_ns_schedule* sch,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Stiefel-manifold step for a contiguous batch of column-orthonormal W (n x k fp32,
+ * n >= k): tangent projection of G (n x k fp32), then the Cayley retraction with
+ * c = lr/2 in Woodbury form (2k x 2k LU with partial pivoting, fp32, no TF32).
+ * W is updated in place; G is read.  n < k returns MUON_ERR_UNSUPPORTED_SHAPE (transpose
+ * the problem, as the page advises).  k <= 4096. */
+MUON_API size_t stiefel_workspace_size(int batch, int n, int k);
+MUON_API muon_status stiefel_cayley_step(float* W, const float* G, int batch, int n, int k, float lr,
+                                void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads the device-side status word of `workspace` into
+ * *status_out (MUON_OK, MUON_ERR_NONFINITE or MUON_ERR_DEVICE_TIMEOUT) and clears it. */
+MUON_API muon_status muon_workspace_device_status(void* workspace, size_t ws_bytes, int* status_out,
+                                         void* stream);
+
+/* Per-kernel-kind device timing, for measurement.  While enabled, every launch is
+ * bracketed by CUDA events on its stream (this adds a little host overhead).
+ * muon_timing_read() synchronises the recorded events and returns, for `kind`, the summed
+ * milliseconds, the launch count and the summed algorithmic work (FLOP for GEMM kinds,
+ * bytes for elementwise kinds) since the last reset. */
+typedef enum {
+    MUON_KERNEL_MOMENTUM = 0,     /* momentum + bf16 cast + Frobenius partial sums        */
+    MUON_KERNEL_SCALE = 1,        /* per-matrix 1 / (||X0|| + eps)                        */
+    MUON_KERNEL_NS_GEMM = 2,      /* tcgen05 Gram / polynomial / apply (bf16, fp32 acc)   */
+    MUON_KERNEL_UPDATE = 3,       /* scale + decoupled weight decay + update              */
+    MUON_KERNEL_SIMT_GEMM = 4,    /* fp32 FMA GEMMs (fp32 NS mode, Stiefel)               */
+    MUON_KERNEL_LU = 5,           /* 2k x 2k LU and triangular solves                     */
+    MUON_KERNEL_MISC = 6,         /* casts, copies, block assembly                        */
+    MUON_KERNEL_KINDS = 7
+} muon_kernel_kind;
+MUON_API muon_status muon_timing_enable(int enable);
+MUON_API muon_status muon_timing_reset(void);
+MUON_API muon_status muon_timing_read(int kind, double* ms, long long* launches, double* work);
+
+MUON_API const char* muon_status_string(muon_status s);
+MUON_API const char* muon_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MUON_B200_H */

@@ -1,0 +1,121 @@
+// Kernel-level interfaces shared by the kernel files and the host orchestration.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace muon {
+
+// Device status bits (first word of every workspace).
+constexpr unsigned kDevErrTimeout = 1u;
+constexpr unsigned kDevErrNonfinite = 2u;
+
+// ------------------------------------------------------------------ tcgen05 grouped GEMM
+// One problem of a grouped launch: out = f * (alpha * (A_op x B_op) + beta * E), f = 1 or
+// (*dscale)^scale_pow, on bf16 operands with fp32 accumulation in TMEM.  A_op is M x K,
+// B_op is K x N; each is read through TMA tensor maps, K-major (contiguous along K) or
+// MN-major (contiguous along M resp. N).  A second ("lo") plane of an operand adds the
+// split-bf16 products hi*lo and lo*hi.  With kSym the output is symmetric: only tiles that
+// reach the upper triangle are computed, and their elements above the diagonal are also
+// stored mirrored.
+constexpr uint32_t kProbAMn = 1u;
+constexpr uint32_t kProbBMn = 2u;
+constexpr uint32_t kProbSym = 4u;
+
+struct alignas(16) TcProblem {
+    const CUtensorMap* tmA[2];
+    const CUtensorMap* tmB[2];
+    const __nv_bfloat16* E[2];
+    __nv_bfloat16* out[2];
+    const float* dscale;
+    int M, N, K;
+    int ld;            // row pitch (elements) of out and E
+    float alpha, beta;
+    int scale_pow;
+    uint32_t flags;
+};
+
+constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64, kTcStages = 4;
+constexpr int kTcThreads = 256;
+// Tile code: problem (12 bits) | m block (10 bits) | n block (10 bits).
+__host__ __device__ inline uint32_t tile_code(int p, int mb, int nb) {
+    return (static_cast<uint32_t>(p) << 20) | (static_cast<uint32_t>(mb) << 10) | static_cast<uint32_t>(nb);
+}
+constexpr int kMaxTileProblems = 4096, kMaxTileBlocks = 1024;
+
+size_t tc_gemm_smem_bytes();
+cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, int num_tiles, unsigned* d_status,
+                           int num_sms, cudaStream_t stream);
+
+// ------------------------------------------------------------------ fp32 SIMT grouped GEMM
+// out[m*ld_out + n] = f * (alpha * sum_k A(m,k) B(k,n) + beta * E[m*ld_e + n]),
+// A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn], fp32 FMA (no TF32).
+struct alignas(16) SimtProblem {
+    const float* A;
+    const float* B;
+    const float* E;
+    float* out;
+    const float* dscale;
+    long long sam, sak, sbk, sbn;
+    long long ld_out, ld_e;
+    int M, N, K;
+    float alpha, beta;
+    int scale_pow;
+    int vec_a, vec_b;  // 16-byte vector loads allowed along the contiguous dimension
+};
+constexpr int kSimtBM = 128, kSimtBN = 128, kSimtBK = 8, kSimtThreads = 256;
+cudaError_t simt_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream);
+
+// ------------------------------------------------------------------ elementwise
+// Per matrix of a momentum/cast launch.
+struct alignas(16) MomentumItem {
+    const void* G;       // bf16 or fp32
+    float* M;            // fp32, updated in place (nullable: then X0 = cast(G))
+    void* X0;            // bf16 (or fp32 in fp32 mode)
+    long long n;         // elements
+    long long block0;    // first block index of this matrix
+    int g_f32;           // G dtype
+    int x_f32;           // X0 dtype
+    int vec;             // all pointers 16-byte aligned: 128-bit accesses allowed
+};
+cudaError_t momentum_cast_launch(const MomentumItem* d_items, int count, long long total_blocks, float beta,
+                                 int nesterov, double* d_partials, cudaStream_t stream);
+constexpr int kEwThreads = 256;
+constexpr int kEwElemsPerBlock = 8192;   // 256 threads x 8 elements x 4
+
+// scale[i] = 1 / (sqrt(sum of partials of matrix i) + eps); flags non-finite sums.
+cudaError_t frob_scale_launch(const long long* d_block0, const long long* d_nblocks, int count,
+                              const double* d_partials, float eps, float* d_scale, unsigned* d_status,
+                              cudaStream_t stream);
+
+struct alignas(16) UpdateItem {
+    void* W;             // bf16 or fp32, in place
+    const void* O;       // bf16 or fp32 NS output (natural layout)
+    void* O_out;         // optional copy of f*O (same dtype as O)
+    const float* dscale; // nullable: O is multiplied by *dscale (NS with zero iterations)
+    long long n;
+    long long block0;
+    float decay;         // 1 - lr*wd
+    float step;          // -lr*scale
+    int w_f32;
+    int o_f32;
+    int vec;
+};
+cudaError_t update_launch(const UpdateItem* d_items, int count, long long total_blocks, cudaStream_t stream);
+
+// dst (dtype dst_f32) = f * src (bf16 or fp32), f = *dscale or 1; batched items.
+struct alignas(16) CastItem {
+    const void* src;
+    void* dst;
+    const float* dscale;
+    long long n;
+    long long block0;
+    int src_f32;
+    int dst_f32;
+    int vec;
+};
+cudaError_t cast_launch(const CastItem* d_items, int count, long long total_blocks, cudaStream_t stream);
+
+}  // namespace muon

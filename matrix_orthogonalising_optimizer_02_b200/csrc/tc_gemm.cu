@@ -1,0 +1,334 @@
+// Grouped, persistent, warp-specialised bf16 GEMM on the 5th-generation tensor cores
+// (tcgen05 + TMEM + TMA) for the three products of one Newton-Schulz iteration
+// ("Muon优化器" page, section "Newton-Schulz 迭代": A = X X^T, B = bA + cA^2, X = aX + BX).
+//
+// CTA layout (256 threads, one CTA per SM):
+//   warp 0 lane 0 : TMA producer -- fills a 4-stage ring of (128 x 64 A, 256 x 64 B) bf16
+//                   tiles, 128-byte swizzled, K-major or MN-major per problem
+//   warp 1 lane 0 : MMA issuer   -- tcgen05.mma 128x256x16 into one of two TMEM
+//                   accumulators (2 x 256 fp32 columns), commits free smem stages
+//   warp 2        : allocates / frees the 512 TMEM columns
+//   warps 4..7    : epilogue     -- tcgen05.ld of its 32-lane quarter, alpha/beta/scale
+//                   epilogue in fp32, bf16 (hi, lo) stores, mirrored stores for symmetric
+//                   outputs; releases the accumulator to the MMA warp
+// Tiles of all problems of a stage come from one list; CTA b takes tiles b, b + grid, ...
+#include <cstdio>
+
+#include "kernels.cuh"
+#include "ptx_sm100.cuh"
+
+namespace muon {
+namespace {
+
+constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
+constexpr int A_BYTES = BM * BK * 2;      // 16 KB
+constexpr int B_BYTES = BN * BK * 2;      // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;   // one 64(MN) x 64(K) box: 8 KB
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COLS = 256;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+
+struct TileInfo {
+    int p, m0, n0;
+};
+__device__ __forceinline__ TileInfo decode(uint32_t code) {
+    TileInfo t;
+    t.p = static_cast<int>(code >> 20);
+    t.m0 = static_cast<int>((code >> 10) & 1023u) * BM;
+    t.n0 = static_cast<int>(code & 1023u) * BN;
+    return t;
+}
+
+// Segments of the K loop: (A plane, B plane) = (hi,hi), then (hi,lo), (lo,hi) when present.
+__device__ __forceinline__ int num_segments(const TcProblem& P) {
+    return 1 + (P.tmB[1] != nullptr) + (P.tmA[1] != nullptr);
+}
+__device__ __forceinline__ void segment_planes(const TcProblem& P, int seg, int& pa, int& pb) {
+    pa = 0;
+    pb = 0;
+    if (seg == 1) {
+        if (P.tmB[1] != nullptr) pb = 1; else pa = 1;
+    } else if (seg == 2) {
+        pa = 1;
+    }
+}
+
+__device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]);
+    w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]);
+    w.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(dst) = w;
+}
+__device__ __forceinline__ void load_bf16x8_add(const __nv_bfloat16* src, float* e) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src));
+    e[0] += bf16_lo_to_f32(w.x); e[1] += bf16_hi_to_f32(w.x);
+    e[2] += bf16_lo_to_f32(w.y); e[3] += bf16_hi_to_f32(w.y);
+    e[4] += bf16_lo_to_f32(w.z); e[5] += bf16_hi_to_f32(w.z);
+    e[6] += bf16_lo_to_f32(w.w); e[7] += bf16_hi_to_f32(w.w);
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__ tiles, int num_tiles,
+               unsigned* dev_status) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* full_bar = bars;
+    uint64_t* empty_bar = bars + STAGES;
+    uint64_t* tfull_bar = bars + 2 * STAGES;
+    uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 128);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------------ TMA producer
+        uint32_t stage = 0, phase = 0;
+        int last_p = -1;
+        bool ok = true;
+        int issued_parity[STAGES];
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode(tiles[t]);
+            const TcProblem& P = probs[ti.p];
+            if (ti.p != last_p) {
+                for (int i = 0; i < 2; ++i) {
+                    if (P.tmA[i]) tmap_acquire(P.tmA[i]);
+                    if (P.tmB[i]) tmap_acquire(P.tmB[i]);
+                }
+                last_p = ti.p;
+            }
+            const bool a_mn = (P.flags & kProbAMn) != 0;
+            const bool b_mn = (P.flags & kProbBMn) != 0;
+            const int kblocks = (P.K + BK - 1) / BK;
+            const int nseg = num_segments(P);
+            for (int seg = 0; seg < nseg && ok; ++seg) {
+                int pa, pb;
+                segment_planes(P, seg, pa, pb);
+                const CUtensorMap* ta = P.tmA[pa];
+                const CUtensorMap* tb = P.tmB[pb];
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, dev_status)) { ok = false; break; }
+                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    const int k0 = kb * BK;
+                    mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+                    issued_parity[stage] = static_cast<int>(phase);
+                    if (!a_mn) {
+                        tma_load_2d(sa, ta, &full_bar[stage], k0, ti.m0);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < BM / 64; ++c)
+                            tma_load_2d(sa + c * MN_CHUNK_BYTES, ta, &full_bar[stage], ti.m0 + 64 * c, k0);
+                    }
+                    if (!b_mn) {
+                        tma_load_2d(sb, tb, &full_bar[stage], k0, ti.n0);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < BN / 64; ++c)
+                            tma_load_2d(sb + c * MN_CHUNK_BYTES, tb, &full_bar[stage], ti.n0 + 64 * c, k0);
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+        }
+        if (!ok) {
+            // Let copies already issued land before the CTA exits (bounded).
+            for (int s = 0; s < STAGES; ++s) {
+                if (issued_parity[s] < 0) continue;
+                const unsigned long long t0 = global_ns();
+                while (!mbar_try_wait(&full_bar[s], static_cast<uint32_t>(issued_parity[s])) &&
+                       global_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------------------ MMA issuer
+        uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+            const TileInfo ti = decode(tiles[t]);
+            const TcProblem& P = probs[ti.p];
+            const bool a_mn = (P.flags & kProbAMn) != 0;
+            const bool b_mn = (P.flags & kProbBMn) != 0;
+            const uint32_t idesc = idesc_bf16_f32(BM, BN, a_mn, b_mn);
+            const int kblocks = (P.K + BK - 1) / BK;
+            const int nseg = num_segments(P);
+            if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, dev_status)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+            uint32_t accumulate = 0;
+            for (int seg = 0; seg < nseg && ok; ++seg) {
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, abort_flag, dev_status)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t base_a = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t base_b = base_a + A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = a_mn ? smem_desc_sw128(base_a + k * 2048, MN_CHUNK_BYTES, 1024)
+                                                 : smem_desc_sw128(base_a + k * 32, 16, 1024);
+                        const uint64_t bd = b_mn ? smem_desc_sw128(base_b + k * 2048, MN_CHUNK_BYTES, 1024)
+                                                 : smem_desc_sw128(base_b + k * 32, 16, 1024);
+                        tc_mma_bf16(d_tmem, ad, bd, idesc, accumulate);
+                        accumulate = 1;
+                    }
+                    tc_commit(&empty_bar[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            tc_commit(&tfull_bar[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        if (!ok) {
+            // Drain: wait (bounded) until every MMA issued so far has finished.
+            tc_commit(&tfull_bar[acc]);
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(&tfull_bar[acc], acc_phase) && global_ns() - t0 < 100000000ull) {
+            }
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        uint32_t acc = 0, acc_phase = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            const TileInfo ti = decode(tiles[t]);
+            const TcProblem& P = probs[ti.p];
+            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status)) break;
+            tc_fence_after();
+            float f = 1.0f;
+            if (P.dscale != nullptr && P.scale_pow > 0) {
+                const float s = __ldg(P.dscale);
+                f = (P.scale_pow == 1) ? s : s * s;
+            }
+            const float alpha = P.alpha * f;
+            const float beta = P.beta * f;
+            const bool sym = (P.flags & kProbSym) != 0;
+            const int row = ti.m0 + q * 32 + lane;
+            const bool row_ok = row < P.M;
+            const bool has_e = (beta != 0.0f) && (P.E[0] != nullptr);
+            const bool lo_out = P.out[1] != nullptr;
+            const uint32_t t_row = tmem_base + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int col0 = ti.n0 + c * 32;
+                if (col0 >= P.N) break;  // uniform across the warp
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(t_row + c * 32, r);
+                tmem_ld_wait();
+                // Rows whose whole chunk lies below the diagonal store nothing.
+                const bool any_store = row_ok && (!sym || col0 + 31 > row - 1);
+                float v[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
+                if (has_e && any_store) {
+                    const size_t base = static_cast<size_t>(row) * P.ld + col0;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        if (col0 + 8 * g < P.N) {
+                            float e[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                            load_bf16x8_add(P.E[0] + base + 8 * g, e);
+                            if (P.E[1] != nullptr) load_bf16x8_add(P.E[1] + base + 8 * g, e);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) v[8 * g + j] = fmaf(beta, e[j], v[8 * g + j]);
+                        }
+                    }
+                }
+                float lo[32];
+                if (lo_out) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) lo[j] = v[j] - __bfloat162float(__float2bfloat16_rn(v[j]));
+                }
+                if (any_store) {
+                    const size_t base = static_cast<size_t>(row) * P.ld + col0;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int cg = col0 + 8 * g;
+                        if (cg >= P.N) continue;
+                        if (!sym || cg >= row) {
+                            store_bf16x8(P.out[0] + base + 8 * g, v + 8 * g);
+                            if (lo_out) store_bf16x8(P.out[1] + base + 8 * g, lo + 8 * g);
+                        } else if (cg + 7 >= row) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                if (cg + j >= row) {
+                                    P.out[0][base + 8 * g + j] = __float2bfloat16_rn(v[8 * g + j]);
+                                    if (lo_out) P.out[1][base + 8 * g + j] = __float2bfloat16_rn(lo[8 * g + j]);
+                                }
+                            }
+                        }
+                    }
+                }
+                if (sym) {
+                    // Mirror: element (row, col) with col > row also goes to (col, row).  For a
+                    // fixed col the 32 lanes write 32 consecutive rows: one 64-byte segment.
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int col = col0 + j;
+                        if (row_ok && col > row && col < P.N) {
+                            const size_t off = static_cast<size_t>(col) * P.ld + row;
+                            P.out[0][off] = __float2bfloat16_rn(v[j]);
+                            if (lo_out) P.out[1][off] = __float2bfloat16_rn(lo[j]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty_bar[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+}  // namespace
+
+size_t tc_gemm_smem_bytes() { return SMEM_TOTAL; }
+
+cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, int num_tiles, unsigned* d_status,
+                           int num_sms, cudaStream_t stream) {
+    if (num_tiles <= 0) return cudaSuccess;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int grid = num_tiles < num_sms ? num_tiles : num_sms;
+    tc_gemm_kernel<<<grid, kTcThreads, SMEM_TOTAL, stream>>>(d_probs, d_tiles, num_tiles, d_status);
+    return cudaGetLastError();
+}
+
+}  // namespace muon
