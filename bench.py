@@ -1,0 +1,309 @@
+"""Benchmark: one full Muon optimizer step on the Llama-7B-shaped parameter set.
+
+Workload: 32 layers x {4 x 4096x4096, 2 x 4096x11008, 11008x4096} = 224 matrices,
+6.476e9 parameters; bf16 weights ~ N(0, 0.02^2), bf16 gradients ~ N(0, 1e-3^2), fp32
+momentum (zero at start); beta 0.95, lr 0.02, weight decay 0.1, Moonlight scale, 5
+Newton-Schulz iterations with (3.4445, -4.7750, 2.0315).  A step is momentum + cast +
+Frobenius scale + 15 grouped tcgen05 GEMM launches + update for all 224 matrices, through
+the C ABI (muon_step_batched).  Synthetic data drawn on the device from a seeded
+generator; the set (52 GB) is far larger than L2, so no flush is needed.
+
+Multi-GPU (torchrun): every rank runs its own full parameter set (the step has no
+exchange), value = ms per parameter set over the whole job, max over ranks.
+`--impl reference` times the fp64 CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+KJ = (3.4445, -4.7750, 2.0315)
+LR, BETA, WD = 0.02, 0.95, 0.1
+WORKLOAD = "llama7b_muon_step"
+
+
+LAYERS = 32
+
+
+def set_shapes():
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    return workloads.llama7b_shapes(LAYERS)
+
+
+def ns_flops_algorithmic(rows, cols, iters=5):
+    """Symmetry-aware count per matrix: X X^T = r^2 s, A A = r^3, B X = 2 r^2 s per iteration."""
+    r, s = min(rows, cols), max(rows, cols)
+    return iters * (3.0 * r * r * s + float(r) ** 3)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        th = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if th:
+            return int(max(th))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(iters):
+    """fp64 oracle Muon step on one 4096x4096 matrix of the set (momentum, `iters` NS
+    iterations, update); returns (seconds, NS FLOP of the sample)."""
+    import numpy as np
+    import oracle as orc
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    r = workloads.rng(1005)
+    W = orc.round_to_bf16(r.standard_normal((4096, 4096)) * 0.02)
+    G = orc.round_to_bf16(r.standard_normal((4096, 4096)) * 1e-3)
+    M = np.zeros_like(G)
+    t0 = time.perf_counter()
+    orc.muon_step(W, G, M, lr=LR, beta=BETA, weight_decay=WD, schedule=orc.fixed_schedule(iters))
+    return time.perf_counter() - t0, ns_flops_algorithmic(4096, 4096, iters)
+
+
+def set_flops():
+    return sum(ns_flops_algorithmic(r, c) for (r, c) in set_shapes())
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "200", "-i", str(self.dev)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait()
+        self.f.flush()
+        rows = [ln.split(",") for ln in open(self.f.name).read().strip().splitlines() if ln.strip()]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows if len(r) >= 9 for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on this host's cores: each step is one bounded sample (one
+    4096x4096 matrix: momentum, one NS iteration, update), extrapolated to the full set by
+    algorithmic NS FLOPs."""
+    if rank != 0:
+        return
+    total = set_flops()
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, fl = oracle_sample(1)
+        if i >= args.warmup:
+            times.append(dt * total / fl)
+    ms = 1e3 * statistics.mean(times)
+    sample = "one 4096x4096 matrix of the set per step (momentum, 1 of 5 NS iterations, update), " \
+             "extrapolated to the 224-matrix set by algorithmic NS FLOP"
+    out = {"metric": "Muon full-step ms per param set (Llama-7B-shaped set)", "value": ms, "unit": "ms",
+           "impl": "reference", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": WORKLOAD, "matrices": 224, "params": 6476005376},
+           "cpu_baseline": {"value": ms, "unit": "ms", "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+           "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--layers", type=int, default=32,
+                    help="Llama-7B layers in the set (32 = the full set; 1 = a profiling-sized case)")
+    args = ap.parse_args()
+    global LAYERS
+    LAYERS = args.layers
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from matrix_orthogonalising_optimizer_02_b200 import binding as mb
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    shapes = set_shapes()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1005 + 7919 * rank)
+    mats = []
+    for (rows, cols) in shapes:
+        W = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda").normal_(0.0, 0.02, generator=gen)
+        G = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda").normal_(0.0, 1e-3, generator=gen)
+        M = torch.zeros((rows, cols), dtype=torch.float32, device="cuda")
+        mats.append(mb.Matrix(W, G, M))
+    hp = mb.hyper(lr=LR, beta=BETA, weight_decay=WD, scale_mode="moonlight", schedule=mb.Schedule.fixed(5, KJ))
+    ws = mb.workspace(mb.muon_step_workspace_size(mats, hp))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        mb.muon_step_batched(mats, hp, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert mb.device_status(ws) == mb.MUON_OK
+
+    # per-kernel-kind device times (events around every launch, on the launching stream)
+    mb.timing_reset()
+    mb.timing_enable(True)
+    n_prof = 2
+    for _ in range(n_prof):
+        step()
+    torch.cuda.synchronize()
+    mb.timing_enable(False)
+    prof = {k: mb.timing_read(k) for k in mb.KERNEL_KINDS}
+    launches_per_step = sum(v[1] for v in prof.values()) / n_prof
+
+    # timed region
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_step = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    assert mb.device_status(ws) == mb.MUON_OK
+
+    # end to end through the public API from host buffers: pinned gradients copied in each step,
+    # the step's device status word read back
+    g_host = [m.G.cpu().pin_memory() for m in mats]
+    h2d = sum(g.numel() * g.element_size() for g in g_host)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.e2e_steps):
+        for m, g in zip(mats, g_host):
+            m.G.copy_(g, non_blocking=True)
+        step()
+        st = mb.device_status(ws, stream)
+        assert st == mb.MUON_OK
+    t1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = t0.elapsed_time(t1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    del g_host
+
+    hbm, tf_burst, tf_sust, peak_src = peaks()
+    ns_ms, ns_launches, ns_flops = prof["ns_gemm"]
+    ns_tflops = ns_flops / (ns_ms * 1e-3) / 1e12
+    mom_ms, _, mom_bytes = prof["momentum"]
+    upd_ms, _, upd_bytes = prof["update"]
+    ew_gbs = (mom_bytes + upd_bytes) / ((mom_ms + upd_ms) * 1e-3) / 1e9
+    total_flops = set_flops()
+    step_ns_share = ns_ms / n_prof / ms_step
+
+    out = {
+        "metric": "Muon full-step ms per param set (Llama-7B-shaped set)",
+        "value": ms_step / world,
+        "unit": "ms",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded on-device normal draws, Llama-7B shapes)",
+        "config": {"workload": WORKLOAD if LAYERS == 32 else f"{WORKLOAD}_{LAYERS}layer", "matrices": len(shapes), "params": sum(r * c for r, c in shapes),
+                   "ns_iters": 5, "coeffs": list(KJ), "lr": LR, "beta": BETA, "weight_decay": WD,
+                   "scale": "moonlight", "l2": "inputs (52 GB) larger than L2; no flush"},
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "matrices_per_s": len(shapes) * world / (ms_step * 1e-3),
+        "ns_tflops": ns_tflops,
+        "ns_frac_of_bf16_peak": ns_tflops / tf_sust,
+        "ns_share_of_step": step_ns_share,
+        "elementwise_gbs": ew_gbs,
+        "elementwise_frac_of_hbm": ew_gbs / hbm,
+        "momentum_gbs": mom_bytes / (mom_ms * 1e-3) / 1e9 if mom_ms else None,
+        "update_gbs": upd_bytes / (upd_ms * 1e-3) / 1e9 if upd_ms else None,
+        "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel (NS Gram/polynomial/apply)",
+                     "achieved": ns_tflops, "peak": tf_sust, "unit": "TFLOP/s", "frac": ns_tflops / tf_sust,
+                     "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                     "work_per_launch": ns_flops / max(ns_launches, 1), "traffic": None},
+        "e2e": {"value": e2e_ms / world, "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
+        "clocks": clk,
+        "total_ns_flops_per_set": total_flops,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl = oracle_sample(5)
+        out["cpu_baseline"] = {"value": 1e3 * dt * total_flops / fl, "unit": "ms", "cores": cpu_cores(),
+                               "kind": "oracle",
+                               "sample": "one 4096x4096 matrix, full step (momentum, 5 NS iterations, update) "
+                                         f"in {dt:.1f} s, extrapolated to the set by algorithmic NS FLOP"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

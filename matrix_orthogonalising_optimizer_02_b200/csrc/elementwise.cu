@@ -156,6 +156,11 @@ update_kernel(const UpdateItem* __restrict__ items, int count) {
             load8(it.O, e, it.o_f32, o);
 #pragma unroll
             for (int j = 0; j < VEC; ++j) o[j] *= f;
+            // A scaled O keeps its storage precision (the page's X /= norm leaves X in bf16).
+            if (it.dscale != nullptr && !it.o_f32) {
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) o[j] = __bfloat162float(__float2bfloat16_rn(o[j]));
+            }
             if (it.O_out != nullptr) {
                 float oc[VEC];
 #pragma unroll
@@ -168,7 +173,8 @@ update_kernel(const UpdateItem* __restrict__ items, int count) {
         } else if (e < it.n) {
             const long long end = e + VEC < it.n ? e + VEC : it.n;
             for (long long k = e; k < end; ++k) {
-                const float o = f * load1(it.O, k, it.o_f32);
+                float o = f * load1(it.O, k, it.o_f32);
+                if (it.dscale != nullptr && !it.o_f32) o = __bfloat162float(__float2bfloat16_rn(o));
                 if (it.O_out != nullptr) store1(it.O_out, k, it.o_f32, o);
                 store1(it.W, k, it.w_f32, fmaf(it.step, o, it.decay * load1(it.W, k, it.w_f32)));
             }

@@ -37,7 +37,7 @@ struct alignas(16) TcProblem {
     uint32_t flags;
 };
 
-constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64, kTcStages = 4;
+constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64, kTcStages = 6;   // pair (2-CTA) tile
 constexpr int kTcThreads = 256;
 // Tile code: problem (12 bits) | m block (10 bits) | n block (10 bits).
 __host__ __device__ inline uint32_t tile_code(int p, int mb, int nb) {
@@ -49,14 +49,15 @@ size_t tc_gemm_smem_bytes();
 cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, int num_tiles, unsigned* d_status,
                            int num_sms, cudaStream_t stream);
 
-// ------------------------------------------------------------------ fp32 SIMT grouped GEMM
+// ------------------------------------------------------------------ SIMT grouped GEMM
 // out[m*ld_out + n] = f * (alpha * sum_k A(m,k) B(k,n) + beta * E[m*ld_e + n]),
-// A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn], fp32 FMA (no TF32).
+// A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn], on the FMA pipes (no TF32).  Each
+// of A, B, E, out is fp32 or fp64 (flags); the accumulator type is chosen per launch.
 struct alignas(16) SimtProblem {
-    const float* A;
-    const float* B;
-    const float* E;
-    float* out;
+    const void* A;
+    const void* B;
+    const void* E;
+    void* out;
     const float* dscale;
     long long sam, sak, sbk, sbn;
     long long ld_out, ld_e;
@@ -64,9 +65,11 @@ struct alignas(16) SimtProblem {
     float alpha, beta;
     int scale_pow;
     int vec_a, vec_b;  // 16-byte vector loads allowed along the contiguous dimension
+    int a_f64, b_f64, e_f64, out_f64;
 };
 constexpr int kSimtBM = 128, kSimtBN = 128, kSimtBK = 8, kSimtThreads = 256;
-cudaError_t simt_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream);
+cudaError_t simt_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream,
+                             bool f64_acc = false);
 
 // ------------------------------------------------------------------ elementwise
 // Per matrix of a momentum/cast launch.

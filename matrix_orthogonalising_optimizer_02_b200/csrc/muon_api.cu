@@ -132,7 +132,9 @@ struct TmapPool {
     }
 };
 
-constexpr int kBoxK128 = kTcBM, kBoxK256 = kTcBN, kBoxMN = 64;
+// TMA boxes: 64 bf16 (128 B) of the contiguous dimension x 128 rows (K-major operand half
+// of a pair tile), or 64 x 64 (one MN-major chunk).
+constexpr int kBoxK = kTcBM / 2, kBoxMN = 64;
 
 // ---------------------------------------------------------------- NS chain (bf16, tcgen05)
 // Appends the 3T grouped launches; returns per matrix the buffer holding the final X.
@@ -167,7 +169,7 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                 void* xin0 = m.X[cur][0];
                 void* xin1 = in_lo ? m.X[cur][1] : nullptr;
                 if (stage == 0) {  // A = X X^T (wide) or X^T X (tall)
-                    const int box_a = m.tall ? kBoxMN : kBoxK128, box_b = m.tall ? kBoxMN : kBoxK256;
+                    const int box_a = m.tall ? kBoxMN : kBoxK, box_b = box_a;
                     P.tmA[0] = pool.get(xin0, m.rows, m.cols, box_a);
                     P.tmA[1] = pool.get(xin1, m.rows, m.cols, box_a);
                     P.tmB[0] = pool.get(xin0, m.rows, m.cols, box_b);
@@ -182,10 +184,10 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                     flops += static_cast<double>(r) * r * s;
                 } else if (stage == 1) {  // B = b A + c A A  (A A = A A^T, A symmetric)
                     void* a1 = split ? m.A[1] : nullptr;
-                    P.tmA[0] = pool.get(m.A[0], r, r, kBoxK128);
-                    P.tmA[1] = pool.get(a1, r, r, kBoxK128);
-                    P.tmB[0] = pool.get(m.A[0], r, r, kBoxK256);
-                    P.tmB[1] = pool.get(a1, r, r, kBoxK256);
+                    P.tmA[0] = pool.get(m.A[0], r, r, kBoxK);
+                    P.tmA[1] = pool.get(a1, r, r, kBoxK);
+                    P.tmB[0] = P.tmA[0];
+                    P.tmB[1] = P.tmA[1];
                     P.E[0] = static_cast<const __nv_bfloat16*>(m.A[0]);
                     P.E[1] = static_cast<const __nv_bfloat16*>(a1);
                     P.out[0] = static_cast<__nv_bfloat16*>(m.B[0]);
@@ -197,16 +199,16 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                 } else {  // X' = a X + B X (wide) or a X + X B (tall)
                     void* b1 = split ? m.B[1] : nullptr;
                     if (!m.tall) {
-                        P.tmA[0] = pool.get(m.B[0], r, r, kBoxK128);
-                        P.tmA[1] = pool.get(b1, r, r, kBoxK128);
+                        P.tmA[0] = pool.get(m.B[0], r, r, kBoxK);
+                        P.tmA[1] = pool.get(b1, r, r, kBoxK);
                         P.tmB[0] = pool.get(xin0, m.rows, m.cols, kBoxMN);
                         P.tmB[1] = pool.get(xin1, m.rows, m.cols, kBoxMN);
                         P.flags = kProbBMn;
                     } else {
-                        P.tmA[0] = pool.get(xin0, m.rows, m.cols, kBoxK128);
-                        P.tmA[1] = pool.get(xin1, m.rows, m.cols, kBoxK128);
-                        P.tmB[0] = pool.get(m.B[0], r, r, kBoxK256);
-                        P.tmB[1] = pool.get(b1, r, r, kBoxK256);
+                        P.tmA[0] = pool.get(xin0, m.rows, m.cols, kBoxK);
+                        P.tmA[1] = pool.get(xin1, m.rows, m.cols, kBoxK);
+                        P.tmB[0] = pool.get(m.B[0], r, r, kBoxK);
+                        P.tmB[1] = pool.get(b1, r, r, kBoxK);
                         P.flags = 0;
                     }
                     P.E[0] = static_cast<const __nv_bfloat16*>(xin0);

@@ -2,7 +2,9 @@
 // product of the Stiefel/Woodbury path, where the result must carry fp32 accuracy.
 // 128 x 128 tiles, K-step 8, 256 threads with an 8 x 8 register block each, double-
 // buffered shared memory.  Operands are addressed by (row, column) strides, so transposed
-// operands (W^T G, X^T X) need no copies.
+// operands (W^T G, X^T X) need no copies.  The Acc = double instantiation stages the fp32
+// operands as fp64 and accumulates with DFMA: used for long reductions (K = n) whose
+// rounding would otherwise accumulate sequentially over thousands of terms.
 #include "kernels.cuh"
 
 namespace muon {
@@ -11,15 +13,24 @@ namespace {
 constexpr int BM = kSimtBM, BN = kSimtBN, BK = kSimtBK;
 constexpr int PAD = 4;
 
-struct Frag {
-    float a[4];
-    float b[4];
-};
+__device__ __forceinline__ double ld1(const void* base, long long off, int f64) {
+    return f64 ? __ldg(static_cast<const double*>(base) + off) : static_cast<double>(__ldg(static_cast<const float*>(base) + off));
+}
+__device__ __forceinline__ void ld4(const void* base, long long off, int f64, double (&r)[4]) {
+    if (f64) {
+        const double2 a = __ldg(reinterpret_cast<const double2*>(static_cast<const double*>(base) + off));
+        const double2 b = __ldg(reinterpret_cast<const double2*>(static_cast<const double*>(base) + off) + 1);
+        r[0] = a.x; r[1] = a.y; r[2] = b.x; r[3] = b.y;
+    } else {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + off));
+        r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+    }
+}
 
 // Thread -> element mapping of a tile load.  If the operand is contiguous along K the
 // 256 threads cover 128 rows x 2 quads of K; otherwise 8 K-rows x 32 quads of M (or N).
-__device__ __forceinline__ void load_tile(const float* __restrict__ base, long long s_mn, long long s_k, int mn0,
-                                          int k0, int MN, int K, int vec, int tid, float (&r)[4]) {
+__device__ __forceinline__ void load_tile(const void* __restrict__ base, int f64, long long s_mn, long long s_k,
+                                          int mn0, int k0, int MN, int K, int vec, int tid, double (&r)[4]) {
     const bool k_contig = (s_k == 1);
     int mn, k;
     if (k_contig) {
@@ -29,41 +40,61 @@ __device__ __forceinline__ void load_tile(const float* __restrict__ base, long l
         k = tid >> 5;
         mn = (tid & 31) * 4;
     }
-    const int gm = mn0 + mn, gk = k0 + k;
+    const long long gm = mn0 + mn, gk = k0 + k;
     if (k_contig) {
         if (vec && gm < MN && gk + 3 < K) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(base + gm * s_mn + gk));
-            r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+            ld4(base, gm * s_mn + gk, f64, r);
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) r[i] = (gm < MN && gk + i < K) ? __ldg(base + gm * s_mn + (gk + i) * s_k) : 0.f;
+            for (int i = 0; i < 4; ++i) r[i] = (gm < MN && gk + i < K) ? ld1(base, gm * s_mn + (gk + i) * s_k, f64) : 0.0;
         }
     } else {
         if (vec && gk < K && gm + 3 < MN) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(base + gm * s_mn + gk * s_k));
-            r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+            ld4(base, gm * s_mn + gk * s_k, f64, r);
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) r[i] = (gk < K && gm + i < MN) ? __ldg(base + (gm + i) * s_mn + gk * s_k) : 0.f;
+            for (int i = 0; i < 4; ++i) r[i] = (gk < K && gm + i < MN) ? ld1(base, (gm + i) * s_mn + gk * s_k, f64) : 0.0;
         }
     }
 }
 
-__device__ __forceinline__ void store_tile(float (*s)[BM + PAD], bool k_contig, int tid, const float (&r)[4]) {
+template <class Acc>
+__device__ __forceinline__ void store_tile(Acc (*s)[BM + PAD], bool k_contig, int tid, const double (&r)[4]) {
     if (k_contig) {
         const int mn = tid >> 1, k = (tid & 1) * 4;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) s[k + i][mn] = r[i];
+        for (int i = 0; i < 4; ++i) s[k + i][mn] = static_cast<Acc>(r[i]);
     } else {
         const int k = tid >> 5, mn = (tid & 31) * 4;
-        *reinterpret_cast<float4*>(&s[k][mn]) = make_float4(r[0], r[1], r[2], r[3]);
+        if constexpr (sizeof(Acc) == sizeof(float)) {
+            *reinterpret_cast<float4*>(&s[k][mn]) = make_float4(static_cast<float>(r[0]), static_cast<float>(r[1]),
+                                                                static_cast<float>(r[2]), static_cast<float>(r[3]));
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[k][mn + i] = static_cast<Acc>(r[i]);
+        }
     }
 }
 
+__device__ __forceinline__ void load4(const float* p, float (&v)[4], int o) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[o] = q.x; v[o + 1] = q.y; v[o + 2] = q.z; v[o + 3] = q.w;
+}
+__device__ __forceinline__ void load4(const double* p, double (&v)[8], int o) {
+    const double2 a = *reinterpret_cast<const double2*>(p);
+    const double2 b = *reinterpret_cast<const double2*>(p + 2);
+    v[o] = a.x; v[o + 1] = a.y; v[o + 2] = b.x; v[o + 3] = b.y;
+}
+__device__ __forceinline__ void load4(const float* p, float (&v)[8], int o) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[o] = q.x; v[o + 1] = q.y; v[o + 2] = q.z; v[o + 3] = q.w;
+}
+
+template <class Acc>
 __global__ void __launch_bounds__(kSimtThreads)
 simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restrict__ tiles, int num_tiles) {
-    __shared__ __align__(16) float As[2][BK][BM + PAD];
-    __shared__ __align__(16) float Bs[2][BK][BN + PAD];
+    __shared__ __align__(16) Acc As[2][BK][BM + PAD];
+    __shared__ __align__(16) Acc Bs[2][BK][BN + PAD];
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
 
@@ -75,16 +106,16 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
         const bool a_kc = (P.sak == 1);
         const bool b_kc = (P.sbk == 1);
 
-        float acc[8][8];
+        Acc acc[8][8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+            for (int j = 0; j < 8; ++j) acc[i][j] = Acc(0);
 
-        float ra[4], rb[4];
+        double ra[4], rb[4];
         // A(m, k) = A[m*sam + k*sak]; B(k, n) = B[k*sbk + n*sbn] -> as an (n, k) operand.
-        load_tile(P.A, P.sam, P.sak, m0, 0, P.M, P.K, P.vec_a, tid, ra);
-        load_tile(P.B, P.sbn, P.sbk, n0, 0, P.N, P.K, P.vec_b, tid, rb);
+        load_tile(P.A, P.a_f64, P.sam, P.sak, m0, 0, P.M, P.K, P.vec_a, tid, ra);
+        load_tile(P.B, P.b_f64, P.sbn, P.sbk, n0, 0, P.N, P.K, P.vec_b, tid, rb);
         __syncthreads();  // previous tile's readers are done with buffer 0
         store_tile(As[0], a_kc, tid, ra);
         store_tile(Bs[0], b_kc, tid, rb);
@@ -95,21 +126,20 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
             const int cur = ks & 1;
             const bool more = ks + 1 < ksteps;
             if (more) {
-                load_tile(P.A, P.sam, P.sak, m0, (ks + 1) * BK, P.M, P.K, P.vec_a, tid, ra);
-                load_tile(P.B, P.sbn, P.sbk, n0, (ks + 1) * BK, P.N, P.K, P.vec_b, tid, rb);
+                load_tile(P.A, P.a_f64, P.sam, P.sak, m0, (ks + 1) * BK, P.M, P.K, P.vec_a, tid, ra);
+                load_tile(P.B, P.b_f64, P.sbn, P.sbk, n0, (ks + 1) * BK, P.N, P.K, P.vec_b, tid, rb);
             }
 #pragma unroll
             for (int k = 0; k < BK; ++k) {
-                const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][k][ty * 4]);
-                const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][k][64 + ty * 4]);
-                const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][k][tx * 4]);
-                const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][k][64 + tx * 4]);
-                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                Acc av[8], bv[8];
+                load4(&As[cur][k][ty * 4], av, 0);
+                load4(&As[cur][k][64 + ty * 4], av, 4);
+                load4(&Bs[cur][k][tx * 4], bv, 0);
+                load4(&Bs[cur][k][64 + tx * 4], bv, 4);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+                    for (int j = 0; j < 8; ++j) acc[i][j] = fma(av[i], bv[j], acc[i][j]);
             }
             if (more) {
                 store_tile(As[cur ^ 1], a_kc, tid, ra);
@@ -132,9 +162,16 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
             for (int j = 0; j < 8; ++j) {
                 const int n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
                 if (n >= P.N) continue;
-                float v = alpha * acc[i][j];
-                if (beta != 0.f) v = fmaf(beta, P.E[m * P.ld_e + n], v);
-                P.out[m * P.ld_out + n] = v;
+                Acc v = static_cast<Acc>(alpha) * acc[i][j];
+                if (beta != 0.f) {
+                    const long long eo = static_cast<long long>(m) * P.ld_e + n;
+                    const Acc e = P.e_f64 ? static_cast<Acc>(static_cast<const double*>(P.E)[eo])
+                                          : static_cast<Acc>(static_cast<const float*>(P.E)[eo]);
+                    v = fma(static_cast<Acc>(beta), e, v);
+                }
+                const long long oo = static_cast<long long>(m) * P.ld_out + n;
+                if (P.out_f64) static_cast<double*>(P.out)[oo] = static_cast<double>(v);
+                else static_cast<float*>(P.out)[oo] = static_cast<float>(v);
             }
         }
     }
@@ -142,14 +179,18 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
 
 }  // namespace
 
-cudaError_t simt_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream) {
+cudaError_t simt_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream,
+                             bool f64_acc) {
     if (num_tiles <= 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int per_sm = 2;
+    const int per_sm = f64_acc ? 1 : 2;
     const int grid = num_tiles < sms * per_sm ? num_tiles : sms * per_sm;
-    simt_gemm_kernel<<<grid, kSimtThreads, 0, stream>>>(d_probs, d_tiles, num_tiles);
+    if (f64_acc)
+        simt_gemm_kernel<double><<<grid, kSimtThreads, 0, stream>>>(d_probs, d_tiles, num_tiles);
+    else
+        simt_gemm_kernel<float><<<grid, kSimtThreads, 0, stream>>>(d_probs, d_tiles, num_tiles);
     return cudaGetLastError();
 }
 

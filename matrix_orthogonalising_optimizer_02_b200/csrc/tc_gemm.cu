@@ -2,16 +2,22 @@
 // (tcgen05 + TMEM + TMA) for the three products of one Newton-Schulz iteration
 // ("Muon优化器" page, section "Newton-Schulz 迭代": A = X X^T, B = bA + cA^2, X = aX + BX).
 //
-// CTA layout (256 threads, one CTA per SM):
-//   warp 0 lane 0 : TMA producer -- fills a 4-stage ring of (128 x 64 A, 256 x 64 B) bf16
-//                   tiles, 128-byte swizzled, K-major or MN-major per problem
-//   warp 1 lane 0 : MMA issuer   -- tcgen05.mma 128x256x16 into one of two TMEM
-//                   accumulators (2 x 256 fp32 columns), commits free smem stages
-//   warp 2        : allocates / frees the 512 TMEM columns
-//   warps 4..7    : epilogue     -- tcgen05.ld of its 32-lane quarter, alpha/beta/scale
-//                   epilogue in fp32, bf16 (hi, lo) stores, mirrored stores for symmetric
-//                   outputs; releases the accumulator to the MMA warp
-// Tiles of all problems of a stage come from one list; CTA b takes tiles b, b + grid, ...
+// Two CTAs of a cluster (a pair on two SMs) compute one 256 x 256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): each CTA stages its 128 rows of A
+// and its 128 columns of B, so every SM reads half of B's bytes a 1-SM 128 x 256 tile
+// would; each CTA's TMEM holds its 128 rows x 256 fp32 columns, twice (double buffer).
+// Roles per CTA (256 threads):
+//   warp 0 lane 0 : TMA producer -- 6-stage ring of (128 x 64 A, 128 x 64 B) bf16 tiles,
+//                   128-byte swizzled, K-major or MN-major per problem; the loads of both
+//                   CTAs count on the leader CTA's "full" barrier (.cta_group::2 form)
+//   warp 1 lane 0 : MMA issuer (leader CTA only) -- commits free the stage in both CTAs
+//                   and signal both CTAs' epilogues (commit with a CTA mask)
+//   warp 2        : TMEM allocation / release (pair-wide)
+//   warps 4..7    : epilogue -- tcgen05.ld of its 32-lane quarter, alpha/beta/scale in fp32,
+//                   bf16 (hi, lo) stores, mirrored stores for symmetric outputs, then an
+//                   arrival on the leader's "TMEM empty" barrier
+// No TMA load uses cluster multicast.  Tiles of all problems of a stage come from one list;
+// pair p takes tiles p, p + pairs, ...  Every wait is bounded (ptx_sm100.cuh).
 #include <cstdio>
 
 #include "kernels.cuh"
@@ -21,14 +27,17 @@ namespace muon {
 namespace {
 
 constexpr int BM = kTcBM, BN = kTcBN, BK = kTcBK, STAGES = kTcStages;
-constexpr int A_BYTES = BM * BK * 2;      // 16 KB
-constexpr int B_BYTES = BN * BK * 2;      // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int MN_CHUNK_BYTES = 64 * BK * 2;   // one 64(MN) x 64(K) box: 8 KB
+constexpr int HM = BM / 2, HN = BN / 2;              // per-CTA rows of A / columns of B
+constexpr int A_BYTES = HM * BK * 2;                 // 16 KB
+constexpr int B_BYTES = HN * BK * 2;                 // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // per CTA
+constexpr int PAIR_STAGE_BYTES = 2 * STAGE_BYTES;    // counted on the leader's barrier
+constexpr int MN_CHUNK_BYTES = 64 * BK * 2;          // one 64(MN) x 64(K) box: 8 KB
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+static_assert(HM == 128 && HN == 128, "pair tile is 256 x 256");
 
 struct TileInfo {
     int p, m0, n0;
@@ -71,21 +80,23 @@ __device__ __forceinline__ void load_bf16x8_add(const __nv_bfloat16* src, float*
     e[6] += bf16_lo_to_f32(w.w); e[7] += bf16_hi_to_f32(w.w);
 }
 
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
 tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__ tiles, int num_tiles,
                unsigned* dev_status) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* full_bar = bars;
-    uint64_t* empty_bar = bars + STAGES;
-    uint64_t* tfull_bar = bars + 2 * STAGES;
-    uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+    uint64_t* full_bar = bars;                  // leader: TMA bytes of both CTAs landed
+    uint64_t* empty_bar = bars + STAGES;        // both: MMAs reading the stage are done
+    uint64_t* tfull_bar = bars + 2 * STAGES;    // both: accumulator ready
+    uint64_t* tempty_bar = bars + 2 * STAGES + 2;   // leader: both epilogues drained it
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();   // 0 = leader, 1 = peer
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -94,19 +105,22 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], 128);
+            mbar_init(&tempty_bar[a], 2 * 128);
         }
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 2) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();     // barriers of both CTAs initialised before any remote access
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Leader-CTA addresses (shared::cluster window) of the barriers both CTAs signal.
+    const uint32_t full_leader = mapa_shared(smem_u32(full_bar), 0);
+    const uint32_t tempty_leader = mapa_shared(smem_u32(tempty_bar), 0);
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -116,7 +130,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
         int issued_parity[STAGES];
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int t = pair; t < num_tiles && ok; t += npairs) {
             const TileInfo ti = decode(tiles[t]);
             const TcProblem& P = probs[ti.p];
             if (ti.p != last_p) {
@@ -128,6 +142,8 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             }
             const bool a_mn = (P.flags & kProbAMn) != 0;
             const bool b_mn = (P.flags & kProbBMn) != 0;
+            const int am0 = ti.m0 + HM * static_cast<int>(rank);
+            const int bn0 = ti.n0 + HN * static_cast<int>(rank);
             const int kblocks = (P.K + BK - 1) / BK;
             const int nseg = num_segments(P);
             for (int seg = 0; seg < nseg && ok; ++seg) {
@@ -140,28 +156,31 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
                     const int k0 = kb * BK;
-                    mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-                    issued_parity[stage] = static_cast<int>(phase);
+                    const uint32_t fb = full_leader + stage * 8u;
+                    if (rank == 0) {
+                        mbar_arrive_expect_tx(&full_bar[stage], PAIR_STAGE_BYTES);
+                        issued_parity[stage] = static_cast<int>(phase);
+                    }
                     if (!a_mn) {
-                        tma_load_2d(sa, ta, &full_bar[stage], k0, ti.m0);
+                        tma_load_2d_pair(sa, ta, fb, k0, am0);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < BM / 64; ++c)
-                            tma_load_2d(sa + c * MN_CHUNK_BYTES, ta, &full_bar[stage], ti.m0 + 64 * c, k0);
+                        for (int c = 0; c < HM / 64; ++c)
+                            tma_load_2d_pair(sa + c * MN_CHUNK_BYTES, ta, fb, am0 + 64 * c, k0);
                     }
                     if (!b_mn) {
-                        tma_load_2d(sb, tb, &full_bar[stage], k0, ti.n0);
+                        tma_load_2d_pair(sb, tb, fb, k0, bn0);
                     } else {
 #pragma unroll
-                        for (int c = 0; c < BN / 64; ++c)
-                            tma_load_2d(sb + c * MN_CHUNK_BYTES, tb, &full_bar[stage], ti.n0 + 64 * c, k0);
+                        for (int c = 0; c < HN / 64; ++c)
+                            tma_load_2d_pair(sb + c * MN_CHUNK_BYTES, tb, fb, bn0 + 64 * c, k0);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
         }
-        if (!ok) {
-            // Let copies already issued land before the CTA exits (bounded).
+        if (!ok && rank == 0) {
+            // Let copies already issued land before the pair exits (bounded).
             for (int s = 0; s < STAGES; ++s) {
                 if (issued_parity[s] < 0) continue;
                 const unsigned long long t0 = global_ns();
@@ -170,11 +189,11 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                 }
             }
         }
-    } else if (warp == 1 && lane == 0) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ------------------------------------------------------------ MMA issuer (leader)
         uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int t = pair; t < num_tiles && ok; t += npairs) {
             const TileInfo ti = decode(tiles[t]);
             const TcProblem& P = probs[ti.p];
             const bool a_mn = (P.flags & kProbAMn) != 0;
@@ -198,19 +217,19 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                                                  : smem_desc_sw128(base_a + k * 32, 16, 1024);
                         const uint64_t bd = b_mn ? smem_desc_sw128(base_b + k * 2048, MN_CHUNK_BYTES, 1024)
                                                  : smem_desc_sw128(base_b + k * 32, 16, 1024);
-                        tc_mma_bf16(d_tmem, ad, bd, idesc, accumulate);
+                        tc_mma_bf16_pair(d_tmem, ad, bd, idesc, accumulate);
                         accumulate = 1;
                     }
-                    tc_commit(&empty_bar[stage]);
+                    tc_commit_pair(&empty_bar[stage], 0x3);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            tc_commit(&tfull_bar[acc]);
+            tc_commit_pair(&tfull_bar[acc], 0x3);
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
         if (!ok) {
             // Drain: wait (bounded) until every MMA issued so far has finished.
-            tc_commit(&tfull_bar[acc]);
+            tc_commit_pair(&tfull_bar[acc], 0x3);
             const unsigned long long t0 = global_ns();
             while (!mbar_try_wait(&tfull_bar[acc], acc_phase) && global_ns() - t0 < 100000000ull) {
             }
@@ -219,7 +238,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         uint32_t acc = 0, acc_phase = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+        for (int t = pair; t < num_tiles; t += npairs) {
             const TileInfo ti = decode(tiles[t]);
             const TcProblem& P = probs[ti.p];
             if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status)) break;
@@ -232,7 +251,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const float alpha = P.alpha * f;
             const float beta = P.beta * f;
             const bool sym = (P.flags & kProbSym) != 0;
-            const int row = ti.m0 + q * 32 + lane;
+            const int row = ti.m0 + HM * static_cast<int>(rank) + q * 32 + lane;
             const bool row_ok = row < P.M;
             const bool has_e = (beta != 0.0f) && (P.E[0] != nullptr);
             const bool lo_out = P.out[1] != nullptr;
@@ -245,7 +264,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                 tmem_ld_32x32b_x32(t_row + c * 32, r);
                 tmem_ld_wait();
                 // Rows whose whole chunk lies below the diagonal store nothing.
-                const bool any_store = row_ok && (!sym || col0 + 31 > row - 1);
+                const bool any_store = row_ok && (!sym || col0 + 31 >= row);
                 float v[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
@@ -302,15 +321,15 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                 }
             }
             tc_fence_before();
-            mbar_arrive(&tempty_bar[acc]);
+            mbar_arrive_cluster(tempty_leader + acc * 8u);
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();     // no CTA leaves while its pair may still touch its memory
     tc_fence_after();
-    if (warp == 2) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (warp == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 }  // namespace
@@ -320,14 +339,28 @@ size_t tc_gemm_smem_bytes() { return SMEM_TOTAL; }
 cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, int num_tiles, unsigned* d_status,
                            int num_sms, cudaStream_t stream) {
     if (num_tiles <= 0) return cudaSuccess;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static int max_pairs = 0;
+    if (max_pairs == 0) {
         cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+        cfg.blockDim = dim3(kTcThreads, 1, 1);
+        cfg.dynamicSmemBytes = SMEM_TOTAL;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&clusters, tc_gemm_kernel, &cfg);
+        if (e != cudaSuccess || clusters <= 0) clusters = num_sms / 2;
+        max_pairs = clusters;
     }
-    const int grid = num_tiles < num_sms ? num_tiles : num_sms;
-    tc_gemm_kernel<<<grid, kTcThreads, SMEM_TOTAL, stream>>>(d_probs, d_tiles, num_tiles, d_status);
+    const int pairs = num_tiles < max_pairs ? num_tiles : max_pairs;
+    tc_gemm_kernel<<<2 * pairs, kTcThreads, SMEM_TOTAL, stream>>>(d_probs, d_tiles, num_tiles, d_status);
     return cudaGetLastError();
 }
 
