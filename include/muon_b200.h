@@ -145,6 +145,29 @@ MUON_API size_t stiefel_workspace_size(int batch, int n, int k);
 MUON_API muon_status stiefel_cayley_step(float* W, const float* G, int batch, int n, int k, float lr,
                                 void* workspace, size_t ws_bytes, void* stream);
 
+/* Frobenius pre-scaling without a workspace: X_out[i] = X0[i] / (||X0[i]||_F + eps) for a
+ * contiguous batch of rows x cols matrices, X0 = bf16(X_in) (fp32 X_in when fp32_mode = 1),
+ * written as out_dtype; the same values ns_orthogonalize gives with zero iterations.  If
+ * scale_out (device, batch floats) is not NULL it receives the per-matrix 1/(||X0|| + eps).
+ * There is no counterpart of this entry point on the source pages: it exists for callers
+ * that cannot allocate device memory when they call it -- code running under a framework
+ * whose allocator owns all device memory and cannot hand out a workspace at that point,
+ * or paths where a cudaMalloc is not allowed because it would synchronise the device.
+ * It allocates nothing: its scratch (fp64 block sums and per-matrix scales, 528 KiB) is a
+ * fixed array inside the library, which every GPU that loads the library holds until the
+ * process exits.  The first call on each device looks up that array's device address
+ * (with the device current) and caches it; make that first call before any stream
+ * capture.  Every call shares the array and overwrites it; nothing in it needs to start
+ * at zero (each slot is written before it is read within a call).  Calls that overlap on
+ * the GPU (e.g. on two streams) race on the array and must be ordered by the caller.
+ * Limits: batch <= MUON_STATIC_MAX_BATCH and batch * ceil(rows*cols / 8192) <=
+ * MUON_STATIC_MAX_BLOCKS, else MUON_ERR_UNSUPPORTED_SHAPE.  Pointers need no alignment. */
+#define MUON_STATIC_MAX_BLOCKS 65536
+#define MUON_STATIC_MAX_BATCH 4096
+MUON_API muon_status muon_frobenius_prescale_static(const void* X_in, int in_dtype, void* X_out, int out_dtype,
+                                                    int batch, int rows, int cols, int fp32_mode, float eps,
+                                                    float* scale_out, void* stream);
+
 /* Synchronises `stream`, then reads the device-side status word of `workspace` into
  * *status_out (MUON_OK, MUON_ERR_NONFINITE or MUON_ERR_DEVICE_TIMEOUT) and clears it. */
 MUON_API muon_status muon_workspace_device_status(void* workspace, size_t ws_bytes, int* status_out,

@@ -29,7 +29,7 @@ EXPORTED = (
     "muon_step_workspace_size", "muon_step_workspace_min", "muon_step_batched",
     "ns_workspace_size", "ns_orthogonalize", "stiefel_workspace_size", "stiefel_cayley_step",
     "muon_workspace_device_status", "muon_timing_enable", "muon_timing_reset", "muon_timing_read",
-    "muon_status_string", "muon_build_info",
+    "muon_status_string", "muon_build_info", "muon_frobenius_prescale_static",
 )
 
 
@@ -81,6 +81,8 @@ def _lib():
         "muon_timing_read": (c_int, [c_int, POINTER(c_double), POINTER(c_longlong), POINTER(c_double)]),
         "muon_status_string": (ctypes.c_char_p, [c_int]),
         "muon_build_info": (ctypes.c_char_p, []),
+        "muon_frobenius_prescale_static": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                                   c_float, c_void_p, c_void_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name, None)
@@ -215,6 +217,23 @@ def stiefel_cayley_step(W, G, lr: float, workspace, stream=None):
     st = _lib().stiefel_cayley_step(W.data_ptr(), G.data_ptr(), batch, n, k, float(lr), workspace.data_ptr(),
                                     workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "stiefel_cayley_step")
+
+
+def frobenius_prescale_static(X_in, X_out, fp32_mode: bool = False, eps: float = 1e-7, scale_out=None,
+                              stream=None):
+    """X_out = X0 / (||X0||_F + eps) per matrix without a workspace: the library's fixed
+    internal scratch is used instead (see muon_frobenius_prescale_static in the header)."""
+    if X_in.dim() == 2:
+        batch, (rows, cols) = 1, X_in.shape
+    else:
+        batch, rows, cols = X_in.shape
+    if tuple(X_out.shape) != tuple(X_in.shape):
+        raise ValueError("X_out must have X_in's shape")
+    st = _lib().muon_frobenius_prescale_static(X_in.data_ptr(), _dtype_code(X_in), X_out.data_ptr(),
+                                               _dtype_code(X_out), batch, rows, cols, int(bool(fp32_mode)),
+                                               float(eps), scale_out.data_ptr() if scale_out is not None else None,
+                                               _stream(stream))
+    _check(st, "muon_frobenius_prescale_static")
 
 
 def device_status(workspace, stream=None) -> int:
