@@ -38,7 +38,8 @@ struct alignas(16) TcProblem {
 };
 
 constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64, kTcStages = 6;   // pair (2-CTA) tile
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;            // 4 role warps + 8 epilogue warps
+constexpr int kTcEpilogueThreads = 256;
 // Tile code: problem (12 bits) | m block (10 bits) | n block (10 bits).
 __host__ __device__ inline uint32_t tile_code(int p, int mb, int nb) {
     return (static_cast<uint32_t>(p) << 20) | (static_cast<uint32_t>(mb) << 10) | static_cast<uint32_t>(nb);

@@ -6,16 +6,16 @@
 // tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): each CTA stages its 128 rows of A
 // and its 128 columns of B, so every SM reads half of B's bytes a 1-SM 128 x 256 tile
 // would; each CTA's TMEM holds its 128 rows x 256 fp32 columns, twice (double buffer).
-// Roles per CTA (256 threads):
+// Roles per CTA (384 threads):
 //   warp 0 lane 0 : TMA producer -- 6-stage ring of (128 x 64 A, 128 x 64 B) bf16 tiles,
 //                   128-byte swizzled, K-major or MN-major per problem; the loads of both
 //                   CTAs count on the leader CTA's "full" barrier (.cta_group::2 form)
 //   warp 1 lane 0 : MMA issuer (leader CTA only) -- commits free the stage in both CTAs
 //                   and signal both CTAs' epilogues (commit with a CTA mask)
 //   warp 2        : TMEM allocation / release (pair-wide)
-//   warps 4..7    : epilogue -- tcgen05.ld of its 32-lane quarter, alpha/beta/scale in fp32,
-//                   bf16 (hi, lo) stores, mirrored stores for symmetric outputs, then an
-//                   arrival on the leader's "TMEM empty" barrier
+//   warps 4..11   : epilogue -- tcgen05.ld of its 32-lane quarter and half of the columns,
+//                   alpha/beta/scale in fp32, bf16 (hi, lo) stores, mirrored stores for
+//                   symmetric outputs, then an arrival on the leader's "TMEM empty" barrier
 // No TMA load uses cluster multicast.  Tiles of all problems of a stage come from one list;
 // pair p takes tiles p, p + pairs, ...  Every wait is bounded (ptx_sm100.cuh).
 #include <cstdio>
@@ -105,7 +105,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], 2 * 128);
+            mbar_init(&tempty_bar[a], 2 * kTcEpilogueThreads);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -236,13 +236,16 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
+        // 8 warps: warp & 3 selects the TMEM lane quarter (rows), (warp - 4) >> 2 the half of
+        // the 256 columns.  E (the a*X or b*A operand) is prefetched one 32-column chunk
+        // ahead, the first chunk before waiting for the accumulator.
         const int q = warp & 3;
+        const int c_beg = ((warp - 4) >> 2) * (BN / 64);
+        const int c_end = c_beg + BN / 64;
         uint32_t acc = 0, acc_phase = 0;
         for (int t = pair; t < num_tiles; t += npairs) {
             const TileInfo ti = decode(tiles[t]);
             const TcProblem& P = probs[ti.p];
-            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status)) break;
-            tc_fence_after();
             float f = 1.0f;
             if (P.dscale != nullptr && P.scale_pow > 0) {
                 const float s = __ldg(P.dscale);
@@ -254,53 +257,69 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const int row = ti.m0 + HM * static_cast<int>(rank) + q * 32 + lane;
             const bool row_ok = row < P.M;
             const bool has_e = (beta != 0.0f) && (P.E[0] != nullptr);
+            const bool e_lo = has_e && (P.E[1] != nullptr);
             const bool lo_out = P.out[1] != nullptr;
+            const size_t row_base = static_cast<size_t>(row) * P.ld;
+            // E of chunk c for this row (zero where not needed or out of range)
+            auto load_e = [&](int c, uint4 (&eh)[4], uint4 (&el)[4]) {
+                const int col0 = ti.n0 + c * 32;
+                const bool need = has_e && row_ok && col0 < P.N && (!sym || col0 + 31 >= row);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const bool ok = need && (col0 + 8 * g < P.N);
+                    eh[g] = ok ? __ldg(reinterpret_cast<const uint4*>(P.E[0] + row_base + col0 + 8 * g))
+                               : make_uint4(0, 0, 0, 0);
+                    el[g] = (ok && e_lo) ? __ldg(reinterpret_cast<const uint4*>(P.E[1] + row_base + col0 + 8 * g))
+                                         : make_uint4(0, 0, 0, 0);
+                }
+            };
+            uint4 eh[4], el[4];
+            load_e(c_beg, eh, el);
+            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status)) break;
+            tc_fence_after();
             const uint32_t t_row = tmem_base + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = c_beg; c < c_end; ++c) {
                 const int col0 = ti.n0 + c * 32;
                 if (col0 >= P.N) break;  // uniform across the warp
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + c * 32, r);
+                uint4 nh[4], nl[4];
+                if (c + 1 < c_end) load_e(c + 1, nh, nl);
                 tmem_ld_wait();
                 // Rows whose whole chunk lies below the diagonal store nothing.
                 const bool any_store = row_ok && (!sym || col0 + 31 >= row);
                 float v[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = alpha * __uint_as_float(r[j]);
-                if (has_e && any_store) {
-                    const size_t base = static_cast<size_t>(row) * P.ld + col0;
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t hw[4] = {eh[g].x, eh[g].y, eh[g].z, eh[g].w};
+                    const uint32_t lw[4] = {el[g].x, el[g].y, el[g].z, el[g].w};
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        if (col0 + 8 * g < P.N) {
-                            float e[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                            load_bf16x8_add(P.E[0] + base + 8 * g, e);
-                            if (P.E[1] != nullptr) load_bf16x8_add(P.E[1] + base + 8 * g, e);
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) v[8 * g + j] = fmaf(beta, e[j], v[8 * g + j]);
-                        }
+                    for (int h = 0; h < 4; ++h) {
+                        const float e0 = bf16_lo_to_f32(hw[h]) + bf16_lo_to_f32(lw[h]);
+                        const float e1 = bf16_hi_to_f32(hw[h]) + bf16_hi_to_f32(lw[h]);
+                        v[8 * g + 2 * h] = fmaf(beta, e0, alpha * __uint_as_float(r[8 * g + 2 * h]));
+                        v[8 * g + 2 * h + 1] = fmaf(beta, e1, alpha * __uint_as_float(r[8 * g + 2 * h + 1]));
                     }
                 }
-                float lo[32];
-                if (lo_out) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) lo[j] = v[j] - __bfloat162float(__float2bfloat16_rn(v[j]));
-                }
                 if (any_store) {
-                    const size_t base = static_cast<size_t>(row) * P.ld + col0;
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         const int cg = col0 + 8 * g;
                         if (cg >= P.N) continue;
+                        float lo[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            lo[j] = v[8 * g + j] - __bfloat162float(__float2bfloat16_rn(v[8 * g + j]));
                         if (!sym || cg >= row) {
-                            store_bf16x8(P.out[0] + base + 8 * g, v + 8 * g);
-                            if (lo_out) store_bf16x8(P.out[1] + base + 8 * g, lo + 8 * g);
+                            store_bf16x8(P.out[0] + row_base + cg, v + 8 * g);
+                            if (lo_out) store_bf16x8(P.out[1] + row_base + cg, lo);
                         } else if (cg + 7 >= row) {
 #pragma unroll
                             for (int j = 0; j < 8; ++j) {
                                 if (cg + j >= row) {
-                                    P.out[0][base + 8 * g + j] = __float2bfloat16_rn(v[8 * g + j]);
-                                    if (lo_out) P.out[1][base + 8 * g + j] = __float2bfloat16_rn(lo[8 * g + j]);
+                                    P.out[0][row_base + cg + j] = __float2bfloat16_rn(v[8 * g + j]);
+                                    if (lo_out) P.out[1][row_base + cg + j] = __float2bfloat16_rn(lo[j]);
                                 }
                             }
                         }
@@ -314,10 +333,16 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                         const int col = col0 + j;
                         if (row_ok && col > row && col < P.N) {
                             const size_t off = static_cast<size_t>(col) * P.ld + row;
-                            P.out[0][off] = __float2bfloat16_rn(v[j]);
-                            if (lo_out) P.out[1][off] = __float2bfloat16_rn(lo[j]);
+                            const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
+                            P.out[0][off] = hv;
+                            if (lo_out) P.out[1][off] = __float2bfloat16_rn(v[j] - __bfloat162float(hv));
                         }
                     }
+                }
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    eh[g] = nh[g];
+                    el[g] = nl[g];
                 }
             }
             tc_fence_before();
