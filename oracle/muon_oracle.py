@@ -247,3 +247,31 @@ def orthogonality_error(W):
     """max |W^T W - I| (§5.1's check, in max-norm)."""
     W = np.asarray(W, dtype=np.float64)
     return float(np.max(np.abs(W.T @ W - np.eye(W.shape[1]))))
+
+
+# ---------------------------------------------------------------------------
+# MuonCayley optimizer update (mlqm.cn/news/1339166, §3.3 and §4.3)
+# ---------------------------------------------------------------------------
+
+def ema_momentum(M0, G, beta: float):
+    """§3.3 / §4.3 ``buf.mul_(momentum).add_(grad, alpha=1 - momentum)``:
+    M1 = beta*M0 + (1 - beta)*G."""
+    return beta * np.asarray(M0, dtype=np.float64) + (1.0 - beta) * np.asarray(G, dtype=np.float64)
+
+
+def center_columns(M):
+    """§4.3 ``buf - buf.mean(dim=0, keepdim=True)``: subtract each column's mean over the
+    rows.  (The §3.3 prose says row mean; the printed code, which is what runs, takes
+    dim=0 -- the reading this oracle follows.)"""
+    M = np.asarray(M, dtype=np.float64)
+    return M - M.mean(axis=0, keepdims=True)
+
+
+def muon_cayley_step(W, G, M0, lr: float, beta: float, center: bool = True):
+    """One MuonCayley update in the order of §4.3: EMA momentum, centering, tangent
+    projection of the centred momentum, Cayley retraction (Woodbury form).
+    Returns (W1, M1)."""
+    M1 = ema_momentum(M0, G, beta)
+    D = center_columns(M1) if center else M1
+    V = project_tangent(W, D)
+    return cayley_woodbury(W, V, lr), M1

@@ -310,3 +310,39 @@ def test_stiefel_toy_run_stays_on_manifold():
     for _ in range(toy["steps"]):
         W = orc.stiefel_cayley_step(W, r.standard_normal(W.shape), toy["lr"])
     assert orc.orthogonality_error(W) < 1e-12
+
+
+# --------------------------------------------------------------------- MuonCayley
+
+def test_ema_momentum_special_cases():
+    r = workloads.rng(51)
+    M0, G = r.standard_normal((6, 4)), r.standard_normal((6, 4))
+    assert np.array_equal(orc.ema_momentum(M0, G, 0.0), G)
+    assert np.array_equal(orc.ema_momentum(M0, G, 1.0), M0)
+    # a constant gradient is a fixed point of the average
+    assert np.allclose(orc.ema_momentum(G, G, 0.9), G)
+
+
+def test_center_columns_is_the_column_mean_projection():
+    r = workloads.rng(52)
+    M = r.standard_normal((7, 5)) + np.arange(5)          # distinct column offsets
+    C = orc.center_columns(M)
+    assert np.allclose(C.sum(axis=0), 0.0, atol=1e-12)     # every column sums to zero
+    assert np.allclose(orc.center_columns(C), C)           # idempotent
+    assert np.allclose(M - C, np.ones((7, 1)) @ M.mean(axis=0, keepdims=True))   # removes a rank-1 row-constant part
+    assert np.allclose(orc.center_columns(np.ones((7, 1)) @ r.standard_normal((1, 5))), 0.0)
+
+
+def test_muon_cayley_step_stays_on_manifold_and_reduces_to_stiefel_step():
+    r = workloads.rng(53)
+    n, k = 48, 12
+    W = _orth(r, n, k)
+    M = np.zeros((n, k))
+    for _ in range(20):
+        G = r.standard_normal((n, k))
+        W, M = orc.muon_cayley_step(W, G, M, lr=3e-3, beta=0.9)
+    assert orc.orthogonality_error(W) < 1e-12
+    # beta = 0, no centering: exactly the plain projected Cayley step of the gradient
+    G = r.standard_normal((n, k))
+    W1, M1 = orc.muon_cayley_step(W, G, np.zeros((n, k)), lr=0.05, beta=0.0, center=False)
+    assert np.allclose(W1, orc.stiefel_cayley_step(W, G, 0.05), atol=1e-14) and np.array_equal(M1, G)
