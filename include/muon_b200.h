@@ -168,6 +168,19 @@ MUON_API muon_status muon_frobenius_prescale_static(const void* X_in, int in_dty
                                                     int batch, int rows, int cols, int fp32_mode, float eps,
                                                     float* scale_out, void* stream);
 
+/* MuonCayley update ("Muon 在 Stiefel 流形上的精确闭式更新" page, §3.3 and §4.3) for a
+ * contiguous batch of column-orthonormal W (n x k fp32, n >= k):
+ *   M <- beta*M + (1 - beta)*G                       (EMA momentum, M fp32, in place)
+ *   D = M - (column means of M over the n rows)      (center = 1; D = M when center = 0)
+ *   W <- Cayley retraction of W along the tangent projection of D, c = lr/2
+ * The centering follows the page's printed code (mean over dim 0, i.e. each column's mean);
+ * the projection and retraction are those of stiefel_cayley_step, whose workspace size
+ * this entry point shares.  Errors as stiefel_cayley_step, plus INVALID_ARG for a null M,
+ * a non-finite beta or center not in {0, 1}. */
+MUON_API size_t muon_cayley_workspace_size(int batch, int n, int k);
+MUON_API muon_status muon_cayley_step(float* W, const float* G, float* M, int batch, int n, int k, float lr,
+                                      float beta, int center, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reads the device-side status word of `workspace` into
  * *status_out (MUON_OK, MUON_ERR_NONFINITE or MUON_ERR_DEVICE_TIMEOUT) and clears it. */
 MUON_API muon_status muon_workspace_device_status(void* workspace, size_t ws_bytes, int* status_out,

@@ -30,6 +30,7 @@ EXPORTED = (
     "ns_workspace_size", "ns_orthogonalize", "stiefel_workspace_size", "stiefel_cayley_step",
     "muon_workspace_device_status", "muon_timing_enable", "muon_timing_reset", "muon_timing_read",
     "muon_status_string", "muon_build_info", "muon_frobenius_prescale_static",
+    "muon_cayley_workspace_size", "muon_cayley_step",
 )
 
 
@@ -81,6 +82,9 @@ def _lib():
         "muon_timing_read": (c_int, [c_int, POINTER(c_double), POINTER(c_longlong), POINTER(c_double)]),
         "muon_status_string": (ctypes.c_char_p, [c_int]),
         "muon_build_info": (ctypes.c_char_p, []),
+        "muon_cayley_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+        "muon_cayley_step": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_float, c_float, c_int,
+                                     c_void_p, c_size_t, c_void_p]),
         "muon_frobenius_prescale_static": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int,
                                                    c_float, c_void_p, c_void_p]),
     }
@@ -234,6 +238,23 @@ def frobenius_prescale_static(X_in, X_out, fp32_mode: bool = False, eps: float =
                                                float(eps), scale_out.data_ptr() if scale_out is not None else None,
                                                _stream(stream))
     _check(st, "muon_frobenius_prescale_static")
+
+
+def muon_cayley_workspace_size(batch: int, n: int, k: int) -> int:
+    return int(_lib().muon_cayley_workspace_size(batch, n, k))
+
+
+def muon_cayley_step(W, G, M, lr: float, beta: float, workspace, center: bool = True, stream=None):
+    if W.dim() == 2:
+        batch, (n, k) = 1, W.shape
+    else:
+        batch, n, k = W.shape
+    if tuple(G.shape) != tuple(W.shape) or tuple(M.shape) != tuple(W.shape):
+        raise ValueError("G and M must have W's shape")
+    st = _lib().muon_cayley_step(W.data_ptr(), G.data_ptr(), M.data_ptr(), batch, n, k, float(lr), float(beta),
+                                 int(bool(center)), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check(st, "muon_cayley_step")
 
 
 def device_status(workspace, stream=None) -> int:

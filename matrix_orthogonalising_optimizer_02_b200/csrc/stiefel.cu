@@ -56,6 +56,40 @@ __global__ void aug_add_identity_kernel(double* Aug, int n2k, long long ld, long
         a[static_cast<long long>(i) * ld + i] += 1.0;
 }
 
+// MuonCayley momentum (§4.3): M <- beta*M + (1 - beta)*G, elementwise over the batch.
+__global__ void ema_kernel(float* __restrict__ M, const float* __restrict__ G, long long total, float beta) {
+    const float omb = 1.0f - beta;
+    for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x)
+        M[e] = fmaf(beta, M[e], omb * G[e]);
+}
+
+// cm[b][j] = mean over the n rows of column j of M[b] (fp64 sum), one thread per column.
+__global__ void column_mean_kernel(const float* __restrict__ M, double* __restrict__ cm, int n, int k) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    if (j >= k) return;
+    const float* m = M + static_cast<long long>(b) * n * k;
+    double s = 0.0;
+    for (int i = 0; i < n; ++i) s += m[static_cast<long long>(i) * k + j];
+    cm[static_cast<long long>(b) * k + j] = s / n;
+}
+
+// D[b] = M[b] - cm[b] broadcast over rows (or a copy of M when cm is null).
+__global__ void center_kernel(const float* __restrict__ M, const double* __restrict__ cm, float* __restrict__ D,
+                              int n, int k, long long total) {
+    for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        if (cm == nullptr) {
+            D[e] = M[e];
+        } else {
+            const long long b = e / (static_cast<long long>(n) * k);
+            const int j = static_cast<int>(e % k);
+            D[e] = static_cast<float>(static_cast<double>(M[e]) - cm[b * k + j]);
+        }
+    }
+}
+
 // Panel factorisation (partial pivoting) of rows j0..N-1, columns j0..j0+nb-1, held in
 // shared memory.  Records the pivot row of each column in piv (absolute row indices).
 __global__ void __launch_bounds__(1024)
@@ -187,7 +221,7 @@ int lu_panel_width(int N) {
 }
 
 struct StiefelLayout {
-    size_t V, b, S, Aug, piv, table_offset, data_bytes;
+    size_t V, b, S, Aug, piv, cm, table_offset, data_bytes;
 };
 StiefelLayout stiefel_layout(int batch, int n, int k) {
     Arena ar;
@@ -198,6 +232,7 @@ StiefelLayout stiefel_layout(int batch, int n, int k) {
     L.S = ar.take(kk * batch);
     L.Aug = ar.take(static_cast<size_t>(2 * k) * (3 * k) * sizeof(double) * batch);
     L.piv = ar.take(static_cast<size_t>(2 * k) * 4 * batch);
+    L.cm = ar.take(static_cast<size_t>(k) * sizeof(double) * batch);
     L.data_bytes = align_up(ar.used, kAlign);
     L.table_offset = kHeaderBytes + L.data_bytes;
     return L;
@@ -263,6 +298,131 @@ SimtProblem gemm(Mat A, Mat B, void* out, long long ldo, bool o64, const void* E
     return P;
 }
 
+// Appends the projection + Woodbury-Cayley launches for W (batch x n x k) with direction
+// source G (may be the workspace V buffer itself: V = G - W sym(W^T G) is then formed in
+// place, each element read and written by one thread).
+muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, uint8_t* ws, unsigned* d_status,
+                          float* W, const float* G, int batch, int n, int k, float lr, size_t ws_bytes) {
+    float* V = reinterpret_cast<float*>(ws + kHeaderBytes + L.V);
+    float* bb = reinterpret_cast<float*>(ws + kHeaderBytes + L.b);
+    float* S = reinterpret_cast<float*>(ws + kHeaderBytes + L.S);
+    double* Aug = reinterpret_cast<double*>(ws + kHeaderBytes + L.Aug);
+    int* piv = reinterpret_cast<int*>(ws + kHeaderBytes + L.piv);
+    const long long nk = static_cast<long long>(n) * k, kk = static_cast<long long>(k) * k;
+    const int N = 2 * k, ncols = 3 * k;
+    const long long ld = ncols, aug_stride = static_cast<long long>(N) * ncols;
+    const float c = 0.5f * lr;
+    const int B = batch;
+    auto Wm = [&](int i, bool t = false) { return Mat{W + i * nk, k, t, false}; };
+    auto Gm = [&](int i) { return Mat{G + i * nk, k, false, false}; };
+    auto Vm = [&](int i, bool t = false) { return Mat{V + i * nk, k, t, false}; };
+    auto bm = [&](int i) { return Mat{bb + i * nk, k, false, false}; };
+    auto Sm = [&](int i) { return Mat{S + i * kk, k, false, false}; };
+    auto Ai = [&](int i) { return Aug + i * aug_stride; };
+    auto Am = [&](int i, long long off) { return Mat{Ai(i) + off, ld, false, true}; };
+
+    std::vector<SimtProblem> pr;
+    // S = W^T G (fp64 accumulation), then sym(S)
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i, true), Gm(i), S + i * kk, k, false, nullptr, 0, false, k, k, n, 1.f, 0.f));
+    add_gemm(plan, img, pr, true); pr.clear();
+    plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * kk * B, [=](cudaStream_t s) {
+        symmetrize_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(S, k, kk);
+        return cudaGetLastError();
+    }});
+    // V = G - W sym(S)
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Sm(i), V + i * nk, k, false, G + i * nk, k, false, n, k, k, -1.f, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    // fp64 blocks: [0,0] = c P = c W^T V, [0,k] = c Q = c W^T W, [k,0] = -c R = -c V^T V
+    for (int i = 0; i < B; ++i) {
+        pr.push_back(gemm(Wm(i, true), Vm(i), Ai(i), ld, true, nullptr, 0, false, k, k, n, c, 0.f));
+        pr.push_back(gemm(Wm(i, true), Wm(i), Ai(i) + k, ld, true, nullptr, 0, false, k, k, n, c, 0.f));
+        pr.push_back(gemm(Vm(i, true), Vm(i), Ai(i) + k * ld, ld, true, nullptr, 0, false, k, k, n, -c, 0.f));
+    }
+    add_gemm(plan, img, pr, true); pr.clear();
+    // [k,k] = -c P^T
+    plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * kk * B, [=](cudaStream_t s) {
+        aug_neg_transpose_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
+        return cudaGetLastError();
+    }});
+    // b = W - V (cQ) - W (-c P^T)
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, k), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + k), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    // C = I + c B U
+    plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * N * B, [=](cudaStream_t s) {
+        aug_add_identity_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(Aug, N, ld, aug_stride);
+        return cudaGetLastError();
+    }});
+    // y = [W^T b; -V^T b] into the right-hand columns (fp64 accumulation)
+    for (int i = 0; i < B; ++i) {
+        pr.push_back(gemm(Wm(i, true), bm(i), Ai(i) + N, ld, true, nullptr, 0, false, k, k, n, 1.f, 0.f));
+        pr.push_back(gemm(Vm(i, true), bm(i), Ai(i) + k * ld + N, ld, true, nullptr, 0, false, k, k, n, -1.f, 0.f));
+    }
+    add_gemm(plan, img, pr, true); pr.clear();
+    // Gaussian elimination with partial pivoting on [C | y], fp64
+    const int nb = lu_panel_width(N);
+    for (int j0 = 0; j0 < N; j0 += nb) {
+        const int w = std::min(nb, N - j0);
+        const size_t smem = static_cast<size_t>(N - j0) * w * sizeof(double);
+        const double lu_flops = 2.0 * (N - j0) * w * w * B;
+        plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
+            static bool attr = false;
+            if (!attr) {
+                cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
+                attr = true;
+            }
+            lu_panel_kernel<<<B, 1024, smem, s>>>(Aug, ld, aug_stride, N, j0, w, piv, N, d_status);
+            return cudaGetLastError();
+        }});
+        const int right = ncols - (j0 + w);
+        if (right > 0) {
+            plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right * B, [=](cudaStream_t s) {
+                lu_swap_trsm_kernel<<<dim3((right + 127) / 128, B), 128, static_cast<size_t>(w) * w * sizeof(double), s>>>(
+                    Aug, ld, aug_stride, j0, w, ncols, piv, N);
+                return cudaGetLastError();
+            }});
+            if (N - j0 - w > 0) {
+                for (int i = 0; i < B; ++i) {
+                    double* base = Ai(i);
+                    pr.push_back(gemm(Mat{base + (j0 + w) * ld + j0, ld, false, true}, Mat{base + j0 * ld + j0 + w, ld, false, true},
+                                      base + (j0 + w) * ld + j0 + w, ld, true, base + (j0 + w) * ld + j0 + w, ld, true,
+                                      N - j0 - w, right, w, -1.f, 1.f));
+                }
+                add_gemm(plan, img, pr, true); pr.clear();
+            }
+        }
+    }
+    // back substitution U z = y' (fp64)
+    const int nblk = (N + kBackBlock - 1) / kBackBlock;
+    for (int q = nblk - 1; q >= 0; --q) {
+        const int i0 = q * kBackBlock, bs = std::min(kBackBlock, N - i0);
+        plan.steps.push_back({MUON_KERNEL_LU, 1.0 * bs * bs * k * B, [=](cudaStream_t s) {
+            back_diag_kernel<<<dim3((k + 127) / 128, B), 128, 0, s>>>(Aug, ld, aug_stride, i0, bs, N, k);
+            return cudaGetLastError();
+        }});
+        if (i0 > 0) {
+            for (int i = 0; i < B; ++i) {
+                double* base = Ai(i);
+                pr.push_back(gemm(Mat{base + i0, ld, false, true}, Mat{base + i0 * ld + N, ld, false, true}, base + N, ld, true,
+                                  base + N, ld, true, i0, k, bs, -1.f, 1.f));
+            }
+            add_gemm(plan, img, pr, true); pr.clear();
+        }
+    }
+    // W_new = b - c V z_top - c W z_bot, then copy into W
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    const size_t bytes = static_cast<size_t>(nk) * B * sizeof(float);
+    plan.steps.push_back({MUON_KERNEL_MISC, 2.0 * bytes, [=](cudaStream_t s) {
+        return cudaMemcpyAsync(W, bb, bytes, cudaMemcpyDeviceToDevice, s);
+    }});
+    if (L.table_offset + img.bytes.size() > ws_bytes) return MUON_ERR_WORKSPACE_TOO_SMALL;
+    return MUON_OK;
+}
+
 }  // namespace
 }  // namespace muon
 
@@ -294,124 +454,53 @@ muon_status stiefel_cayley_step(float* W, const float* G, int batch, int n, int 
     kw.put(W); kw.put(G); kw.put(batch); kw.put(n); kw.put(k); kw.put(lr); kw.put(ws_bytes);
 
     auto build = [&](Plan& plan, TableImage& img) -> muon_status {
-        float* V = reinterpret_cast<float*>(ws + kHeaderBytes + L.V);
-        float* bb = reinterpret_cast<float*>(ws + kHeaderBytes + L.b);
-        float* S = reinterpret_cast<float*>(ws + kHeaderBytes + L.S);
-        double* Aug = reinterpret_cast<double*>(ws + kHeaderBytes + L.Aug);
-        int* piv = reinterpret_cast<int*>(ws + kHeaderBytes + L.piv);
-        const long long nk = static_cast<long long>(n) * k, kk = static_cast<long long>(k) * k;
-        const int N = 2 * k, ncols = 3 * k;
-        const long long ld = ncols, aug_stride = static_cast<long long>(N) * ncols;
-        const float c = 0.5f * lr;
-        const int B = batch;
-        auto Wm = [&](int i, bool t = false) { return Mat{W + i * nk, k, t, false}; };
-        auto Gm = [&](int i) { return Mat{G + i * nk, k, false, false}; };
-        auto Vm = [&](int i, bool t = false) { return Mat{V + i * nk, k, t, false}; };
-        auto bm = [&](int i) { return Mat{bb + i * nk, k, false, false}; };
-        auto Sm = [&](int i) { return Mat{S + i * kk, k, false, false}; };
-        auto Ai = [&](int i) { return Aug + i * aug_stride; };
-        auto Am = [&](int i, long long off) { return Mat{Ai(i) + off, ld, false, true}; };
+        return build_stiefel(plan, img, L, ws, d_status, W, G, batch, n, k, lr, ws_bytes);
+    };
+    return run_plan(kw.k, workspace, L.table_offset, build, stream);
+}
 
-        std::vector<SimtProblem> pr;
-        // S = W^T G (fp64 accumulation), then sym(S)
-        for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i, true), Gm(i), S + i * kk, k, false, nullptr, 0, false, k, k, n, 1.f, 0.f));
-        add_gemm(plan, img, pr, true); pr.clear();
-        plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * kk * B, [=](cudaStream_t s) {
-            symmetrize_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(S, k, kk);
+size_t muon_cayley_workspace_size(int batch, int n, int k) { return stiefel_workspace_size(batch, n, k); }
+
+muon_status muon_cayley_step(float* W, const float* G, float* M, int batch, int n, int k, float lr, float beta,
+                             int center, void* workspace, size_t ws_bytes, void* stream_) {
+    if (M == nullptr || !std::isfinite(beta) || (center != 0 && center != 1)) return MUON_ERR_INVALID_ARG;
+    if (W == nullptr || G == nullptr || workspace == nullptr) return MUON_ERR_INVALID_ARG;
+    if (batch <= 0 || batch > kMaxTileProblems / 4 || n <= 0 || k <= 0 || !std::isfinite(lr))
+        return MUON_ERR_INVALID_ARG;
+    if (n < k || k > 4096 || n > kMaxTileBlocks * kSimtBM) return MUON_ERR_UNSUPPORTED_SHAPE;
+    if (!al16(W) || !al16(G) || !al16(M) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MUON_ERR_ALIGNMENT;
+    if (ws_bytes < muon_cayley_workspace_size(batch, n, k)) return MUON_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const StiefelLayout L = stiefel_layout(batch, n, k);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    unsigned* d_status = static_cast<unsigned*>(workspace);
+
+    KeyWriter kw;
+    kw.put(4);  // plan kind: MuonCayley
+    kw.put(W); kw.put(G); kw.put(M); kw.put(batch); kw.put(n); kw.put(k); kw.put(lr); kw.put(beta); kw.put(center);
+    kw.put(ws_bytes);
+
+    auto build = [&](Plan& plan, TableImage& img) -> muon_status {
+        float* V = reinterpret_cast<float*>(ws + kHeaderBytes + L.V);
+        double* cm = center ? reinterpret_cast<double*>(ws + kHeaderBytes + L.cm) : nullptr;
+        const long long total = static_cast<long long>(batch) * n * k;
+        const int grid = static_cast<int>(std::min<long long>((total + 255) / 256, 148LL * 16));
+        const float b = beta;
+        plan.steps.push_back({MUON_KERNEL_MOMENTUM, 12.0 * total, [=](cudaStream_t s) {
+            ema_kernel<<<grid, 256, 0, s>>>(M, G, total, b);
             return cudaGetLastError();
         }});
-        // V = G - W sym(S)
-        for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Sm(i), V + i * nk, k, false, G + i * nk, k, false, n, k, k, -1.f, 1.f));
-        add_gemm(plan, img, pr); pr.clear();
-        // fp64 blocks: [0,0] = c P = c W^T V, [0,k] = c Q = c W^T W, [k,0] = -c R = -c V^T V
-        for (int i = 0; i < B; ++i) {
-            pr.push_back(gemm(Wm(i, true), Vm(i), Ai(i), ld, true, nullptr, 0, false, k, k, n, c, 0.f));
-            pr.push_back(gemm(Wm(i, true), Wm(i), Ai(i) + k, ld, true, nullptr, 0, false, k, k, n, c, 0.f));
-            pr.push_back(gemm(Vm(i, true), Vm(i), Ai(i) + k * ld, ld, true, nullptr, 0, false, k, k, n, -c, 0.f));
-        }
-        add_gemm(plan, img, pr, true); pr.clear();
-        // [k,k] = -c P^T
-        plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * kk * B, [=](cudaStream_t s) {
-            aug_neg_transpose_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
-            return cudaGetLastError();
-        }});
-        // b = W - V (cQ) - W (-c P^T)
-        for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, k), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
-        add_gemm(plan, img, pr); pr.clear();
-        for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + k), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
-        add_gemm(plan, img, pr); pr.clear();
-        // C = I + c B U
-        plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * N * B, [=](cudaStream_t s) {
-            aug_add_identity_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(Aug, N, ld, aug_stride);
-            return cudaGetLastError();
-        }});
-        // y = [W^T b; -V^T b] into the right-hand columns (fp64 accumulation)
-        for (int i = 0; i < B; ++i) {
-            pr.push_back(gemm(Wm(i, true), bm(i), Ai(i) + N, ld, true, nullptr, 0, false, k, k, n, 1.f, 0.f));
-            pr.push_back(gemm(Vm(i, true), bm(i), Ai(i) + k * ld + N, ld, true, nullptr, 0, false, k, k, n, -1.f, 0.f));
-        }
-        add_gemm(plan, img, pr, true); pr.clear();
-        // Gaussian elimination with partial pivoting on [C | y], fp64
-        const int nb = lu_panel_width(N);
-        for (int j0 = 0; j0 < N; j0 += nb) {
-            const int w = std::min(nb, N - j0);
-            const size_t smem = static_cast<size_t>(N - j0) * w * sizeof(double);
-            const double lu_flops = 2.0 * (N - j0) * w * w * B;
-            plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
-                static bool attr = false;
-                if (!attr) {
-                    cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
-                    attr = true;
-                }
-                lu_panel_kernel<<<B, 1024, smem, s>>>(Aug, ld, aug_stride, N, j0, w, piv, N, d_status);
+        if (cm != nullptr) {
+            plan.steps.push_back({MUON_KERNEL_MISC, 4.0 * total, [=](cudaStream_t s) {
+                column_mean_kernel<<<dim3((k + 127) / 128, batch), 128, 0, s>>>(M, cm, n, k);
                 return cudaGetLastError();
             }});
-            const int right = ncols - (j0 + w);
-            if (right > 0) {
-                plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right * B, [=](cudaStream_t s) {
-                    lu_swap_trsm_kernel<<<dim3((right + 127) / 128, B), 128, static_cast<size_t>(w) * w * sizeof(double), s>>>(
-                        Aug, ld, aug_stride, j0, w, ncols, piv, N);
-                    return cudaGetLastError();
-                }});
-                if (N - j0 - w > 0) {
-                    for (int i = 0; i < B; ++i) {
-                        double* base = Ai(i);
-                        pr.push_back(gemm(Mat{base + (j0 + w) * ld + j0, ld, false, true}, Mat{base + j0 * ld + j0 + w, ld, false, true},
-                                          base + (j0 + w) * ld + j0 + w, ld, true, base + (j0 + w) * ld + j0 + w, ld, true,
-                                          N - j0 - w, right, w, -1.f, 1.f));
-                    }
-                    add_gemm(plan, img, pr, true); pr.clear();
-                }
-            }
         }
-        // back substitution U z = y' (fp64)
-        const int nblk = (N + kBackBlock - 1) / kBackBlock;
-        for (int q = nblk - 1; q >= 0; --q) {
-            const int i0 = q * kBackBlock, bs = std::min(kBackBlock, N - i0);
-            plan.steps.push_back({MUON_KERNEL_LU, 1.0 * bs * bs * k * B, [=](cudaStream_t s) {
-                back_diag_kernel<<<dim3((k + 127) / 128, B), 128, 0, s>>>(Aug, ld, aug_stride, i0, bs, N, k);
-                return cudaGetLastError();
-            }});
-            if (i0 > 0) {
-                for (int i = 0; i < B; ++i) {
-                    double* base = Ai(i);
-                    pr.push_back(gemm(Mat{base + i0, ld, false, true}, Mat{base + i0 * ld + N, ld, false, true}, base + N, ld, true,
-                                      base + N, ld, true, i0, k, bs, -1.f, 1.f));
-                }
-                add_gemm(plan, img, pr, true); pr.clear();
-            }
-        }
-        // W_new = b - c V z_top - c W z_bot, then copy into W
-        for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
-        add_gemm(plan, img, pr); pr.clear();
-        for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
-        add_gemm(plan, img, pr); pr.clear();
-        const size_t bytes = static_cast<size_t>(nk) * B * sizeof(float);
-        plan.steps.push_back({MUON_KERNEL_MISC, 2.0 * bytes, [=](cudaStream_t s) {
-            return cudaMemcpyAsync(W, bb, bytes, cudaMemcpyDeviceToDevice, s);
+        plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * total, [=](cudaStream_t s) {
+            center_kernel<<<grid, 256, 0, s>>>(M, cm, V, n, k, total);
+            return cudaGetLastError();
         }});
-        if (L.table_offset + img.bytes.size() > ws_bytes) return MUON_ERR_WORKSPACE_TOO_SMALL;
-        return MUON_OK;
+        return build_stiefel(plan, img, L, ws, d_status, W, V, batch, n, k, lr, ws_bytes);
     };
     return run_plan(kw.k, workspace, L.table_offset, build, stream);
 }

@@ -77,3 +77,28 @@ def test_stiefel_workload_100_steps():
         mb.stiefel_cayley_step(W, G, lr, ws)
     assert mb.device_status(ws) == mb.MUON_OK
     assert orth_err_dev(W) <= 1e-5
+
+
+@pytest.mark.parametrize("center", [True, False])
+def test_muon_cayley_steps_match_oracle(center):
+    """MuonCayley (EMA momentum, column centering, projection, Cayley) over 5 steps with
+    the page's starting values lr = 3e-3, momentum 0.9."""
+    batch, n, k, lr, beta = 2, 256, 64, 3e-3, 0.9
+    Ws = workloads.stiefel_problem(seed=960, batch=batch, n=n, k=k)
+    W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+    M = torch.zeros_like(W)
+    ws = mb.workspace(mb.muon_cayley_workspace_size(batch, n, k))
+    Wr = [Ws[i].copy() for i in range(batch)]
+    Mr = [np.zeros((n, k)) for _ in range(batch)]
+    for step in range(5):
+        Gs = workloads.stiefel_gradient(960, step, batch, n, k)
+        G = torch.tensor(Gs, dtype=torch.float32, device="cuda")
+        mb.muon_cayley_step(W, G, M, lr, beta, ws, center=center)
+        for i in range(batch):
+            Wr[i], Mr[i] = orc.muon_cayley_step(Wr[i], Gs[i].astype(np.float64), Mr[i], lr, float(np.float32(beta)),
+                                                center=center)
+    assert mb.device_status(ws) == mb.MUON_OK
+    for i in range(batch):
+        assert np.max(np.abs(host(W[i]) - Wr[i])) <= 2e-5
+        assert np.max(np.abs(host(M[i]) - Mr[i])) <= 1e-5 * max(1.0, np.max(np.abs(Mr[i])))
+        assert orc.orthogonality_error(host(W[i])) <= 1e-5
