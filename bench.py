@@ -137,6 +137,79 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def _time_ms(fn, warmup, steps):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def secondary_measurements():
+    """The other parameter sets of the method, each timed on the device (CUDA events,
+    warm-up first): a 64 x 1024^2 low-rank batch through ns_orthogonalize under the fixed and
+    the hybrid schedule, the GPT-2-small set's full step, the 16 x 4096 x 1024 Stiefel step
+    and the single 256 x 128 fp32 step."""
+    import torch
+    from matrix_orthogonalising_optimizer_02_b200 import binding as mb
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    out = {}
+    # low-rank batch
+    X = torch.tensor(workloads.low_rank_plus_noise(batch=64, n=1024)).to(torch.bfloat16).cuda()
+    Y = torch.empty_like(X)
+    for name, sch, iters in [("lowrank64_kj5_split2", mb.Schedule.fixed(5, n_split_iters=2), 5),
+                             ("lowrank64_hybrid_split4", mb.Schedule.hybrid(n_split_iters=4), 10)]:
+        ws = mb.workspace(mb.ns_workspace_size(64, 1024, 1024, sch))
+        ms = _time_ms(lambda: mb.ns_orthogonalize(X, Y, sch, ws), 2, 5)
+        fl = 64 * iters * 4.0 * 1024 ** 3
+        out[name] = {"ms": ms, "algorithmic_tflops": fl / (ms * 1e-3) / 1e12}
+        del ws
+    del X, Y
+    # GPT-2-small set
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1003)
+    mats = []
+    for (rows, cols) in workloads.gpt2_small_shapes(12):
+        mats.append(mb.Matrix(torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda").normal_(0, 0.02, generator=gen),
+                              torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda").normal_(0, 1e-3, generator=gen),
+                              torch.zeros((rows, cols), dtype=torch.float32, device="cuda")))
+    hp = mb.hyper(lr=LR, beta=BETA, weight_decay=WD)
+    ws = mb.workspace(mb.muon_step_workspace_size(mats, hp))
+    ms = _time_ms(lambda: mb.muon_step_batched(mats, hp, ws), 3, 10)
+    fl = sum(ns_flops_algorithmic(r, c) for r, c in workloads.gpt2_small_shapes(12))
+    out["gpt2_small_step"] = {"ms": ms, "ns_algorithmic_tflops": fl / (ms * 1e-3) / 1e12}
+    del mats, ws
+    # Stiefel step
+    W = torch.tensor(workloads.stiefel_problem(batch=16, n=4096, k=1024), dtype=torch.float32, device="cuda")
+    G = torch.empty_like(W).normal_(0, 1.0, generator=gen)
+    ws = mb.workspace(mb.stiefel_workspace_size(16, 4096, 1024))
+    mb.timing_reset()
+    mb.timing_enable(True)
+    mb.stiefel_cayley_step(W, G, 1e-2, ws)
+    torch.cuda.synchronize()
+    mb.timing_enable(False)
+    kinds = {k: mb.timing_read(k) for k in ("simt_gemm", "lu", "misc")}
+    work = kinds["simt_gemm"][2] + kinds["lu"][2]
+    ms = _time_ms(lambda: mb.stiefel_cayley_step(W, G, 1e-2, ws), 1, 3)
+    out["stiefel_16x4096x1024_step"] = {"ms": ms, "fma_tflops": work / (ms * 1e-3) / 1e12,
+                                        "kernel_ms": {k: v[0] for k, v in kinds.items()},
+                                        "simt_gemm_tflops": kinds["simt_gemm"][2] / (kinds["simt_gemm"][0] * 1e-3) / 1e12}
+    del W, G, ws
+    # single fp32 matrix
+    Wn, Gn, Mn = workloads.single_fp32()
+    one = [mb.Matrix(torch.tensor(Wn).cuda(), torch.tensor(Gn).cuda(), torch.tensor(Mn).cuda())]
+    hp1 = mb.hyper(lr=0.02, beta=0.95, weight_decay=0.0, schedule=mb.Schedule.fixed(5, fp32_mode=True))
+    ws = mb.workspace(mb.muon_step_workspace_size(one, hp1))
+    out["single_256x128_fp32_step_us"] = 1e3 * _time_ms(lambda: mb.muon_step_batched(one, hp1, ws), 5, 50)
+    return out
+
+
 def run_reference(args, rank, world):
     """The oracle as it stands, on this host's cores: each step is one bounded sample (one
     4096x4096 matrix: momentum, one NS iteration, update), extrapolated to the full set by
@@ -169,6 +242,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other parameter sets")
     ap.add_argument("--layers", type=int, default=32,
                     help="Llama-7B layers in the set (32 = the full set; 1 = a profiling-sized case)")
     args = ap.parse_args()
@@ -315,6 +389,10 @@ def main():
         "clocks": clk,
         "total_ns_flops_per_set": total_flops,
     }
+    if rank == 0 and world == 1 and not args.no_secondary and LAYERS == 32:
+        del mats, ws
+        torch.cuda.empty_cache()
+        out["secondary"] = secondary_measurements()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, fl = oracle_sample(5)
         out["cpu_baseline"] = {"value": 1e3 * dt * total_flops / fl, "unit": "ms", "cores": cpu_cores(),

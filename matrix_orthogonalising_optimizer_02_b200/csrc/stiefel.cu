@@ -6,7 +6,8 @@
 //              b = W - c U (B W) = W - c V Q + c W P^T,  y = B b = [W^T b; -V^T b]
 //              z = C^-1 y,  W_new = b - c (V z_top + W z_bot)
 // No TF32 anywhere.  The n x k panel products run on the FMA pipes in fp32; the reductions
-// over n (W^T G, the blocks P, Q, R and y) accumulate in fp64.  The augmented 2k x (2k + k)
+// over n (W^T G, the blocks P, Q, R and y) are split into 512-row chunks accumulated in fp32
+// in parallel and summed in fp64.  The augmented 2k x (2k + k)
 // matrix [C | y] is held and eliminated in fp64 (Gaussian elimination with partial
 // pivoting, blocked: panel factorisation in shared memory, row swaps + unit-lower solve on
 // the right-hand columns, rank-nb GEMM update), then blocked back substitution: C has
@@ -88,6 +89,42 @@ __global__ void center_kernel(const float* __restrict__ M, const double* __restr
             D[e] = static_cast<float>(static_cast<double>(M[e]) - cm[b * k + j]);
         }
     }
+}
+
+// out = alpha * sum_j part_j + beta * E, the chunk partials summed in fp64 in order j = 0..
+struct SplitKItem {
+    const float* part;   // nsplit consecutive M x N fp32 partials
+    void* out;
+    const void* E;
+    long long ld_out, ld_e;
+    long long block0;
+    int M, N, nsplit;
+    float alpha, beta;
+    int out_f64, e_f64;
+};
+__global__ void splitk_reduce_kernel(const SplitKItem* __restrict__ items, int count) {
+    const long long b = blockIdx.x;
+    int lo = 0, hi = count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (items[mid].block0 <= b) lo = mid; else hi = mid - 1;
+    }
+    const SplitKItem& it = items[lo];
+    const long long mn = static_cast<long long>(it.M) * it.N;
+    const long long e = (b - it.block0) * blockDim.x + threadIdx.x;
+    if (e >= mn) return;
+    double sum = 0.0;
+    for (int j = 0; j < it.nsplit; ++j) sum += static_cast<double>(it.part[j * mn + e]);
+    const long long m = e / it.N, nn = e % it.N;
+    double v = static_cast<double>(it.alpha) * sum;
+    if (it.beta != 0.f) {
+        const long long eo = m * it.ld_e + nn;
+        v += static_cast<double>(it.beta) *
+             (it.e_f64 ? static_cast<const double*>(it.E)[eo] : static_cast<double>(static_cast<const float*>(it.E)[eo]));
+    }
+    const long long oo = m * it.ld_out + nn;
+    if (it.out_f64) static_cast<double*>(it.out)[oo] = v;
+    else static_cast<float*>(it.out)[oo] = static_cast<float>(v);
 }
 
 // Panel factorisation (partial pivoting) of rows j0..N-1, columns j0..j0+nb-1, held in
@@ -192,6 +229,57 @@ __global__ void lu_swap_trsm_kernel(double* Aug, long long ld, long long stride,
     }
 }
 
+// Within the current block column: apply the row swaps of panel rows j0..j0+w-1 to the
+// earlier multiplier columns [c_lo, c_hi), so the block's L stays consistently permuted.
+__global__ void lu_swap_cols_kernel(double* Aug, long long ld, long long stride, int c_lo, int c_hi, int j0, int w,
+                                    const int* piv, long long piv_stride) {
+    double* a = Aug + blockIdx.y * stride;
+    const int* pv = piv + blockIdx.y * piv_stride;
+    const int c = c_lo + blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= c_hi) return;
+    for (int i = 0; i < w; ++i) {
+        const int p = pv[j0 + i];
+        if (p != j0 + i) {
+            const double t = a[(j0 + static_cast<long long>(i)) * ld + c];
+            a[(j0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
+            a[static_cast<long long>(p) * ld + c] = t;
+        }
+    }
+}
+
+// After a block column J0..J0+JB-1 is factorised: for every column c >= c_lo, apply the
+// block's JB row swaps in order, then solve with the JB x JB unit-lower L11 (U12 = L11^-1 A12).
+constexpr int kLuBlock = 128;
+__global__ void __launch_bounds__(128)
+lu_block_swap_trsm_kernel(double* Aug, long long ld, long long stride, int J0, int JB, int c_lo, int ncols,
+                          const int* piv, long long piv_stride) {
+    extern __shared__ double Lb[];   // JB x JB
+    double* a = Aug + blockIdx.y * stride;
+    const int* pv = piv + blockIdx.y * piv_stride;
+    for (int e = threadIdx.x; e < JB * JB; e += blockDim.x) {
+        const int i = e / JB, j = e % JB;
+        Lb[e] = a[(J0 + static_cast<long long>(i)) * ld + J0 + j];
+    }
+    __syncthreads();
+    const int c = c_lo + blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= ncols) return;
+    for (int i = 0; i < JB; ++i) {
+        const int p = pv[J0 + i];
+        if (p != J0 + i) {
+            const double t = a[(J0 + static_cast<long long>(i)) * ld + c];
+            a[(J0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
+            a[static_cast<long long>(p) * ld + c] = t;
+        }
+    }
+    double x[kLuBlock];
+    for (int i = 0; i < JB; ++i) {
+        double v = a[(J0 + static_cast<long long>(i)) * ld + c];
+        for (int l = 0; l < i; ++l) v = fma(-Lb[i * JB + l], x[l], v);
+        x[i] = v;
+        a[(J0 + static_cast<long long>(i)) * ld + c] = v;
+    }
+}
+
 // Back substitution on one diagonal block: rows i0..i0+bs-1 of the right-hand columns
 // (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows).
 constexpr int kBackBlock = 64;
@@ -221,8 +309,13 @@ int lu_panel_width(int N) {
 }
 
 struct StiefelLayout {
-    size_t V, b, S, Aug, piv, cm, table_offset, data_bytes;
+    size_t V, b, S, Aug, piv, cm, part, table_offset, data_bytes;
 };
+
+// Split-K for the reductions over n: chunks of kSplitK rows summed in fp32, chunk partial
+// sums added in fp64 in a fixed order.
+constexpr int kSplitK = 512;
+int splitk_parts(int n) { return (n + kSplitK - 1) / kSplitK; }
 StiefelLayout stiefel_layout(int batch, int n, int k) {
     Arena ar;
     StiefelLayout L;
@@ -233,6 +326,8 @@ StiefelLayout stiefel_layout(int batch, int n, int k) {
     L.Aug = ar.take(static_cast<size_t>(2 * k) * (3 * k) * sizeof(double) * batch);
     L.piv = ar.take(static_cast<size_t>(2 * k) * 4 * batch);
     L.cm = ar.take(static_cast<size_t>(k) * sizeof(double) * batch);
+    // largest split-K group: the three k x k blocks P, Q, R of every matrix
+    L.part = ar.take(static_cast<size_t>(3) * batch * splitk_parts(n) * k * k * sizeof(float));
     L.data_bytes = align_up(ar.used, kAlign);
     L.table_offset = kHeaderBytes + L.data_bytes;
     return L;
@@ -245,32 +340,90 @@ size_t stiefel_tables_bound(int batch, int n, int k) {
     auto tiles = [](long long M, long long Nn) { return ((M + kSimtBM - 1) / kSimtBM) * ((Nn + kSimtBN - 1) / kSimtBN); };
     long long t = 0;
     t += tiles(k, k) * 1 + tiles(n, k) * 1 + tiles(k, k) * 3 + tiles(n, k) * 2 + tiles(k, k) * 2 + tiles(n, k) * 2;
-    for (int p = 0; p < panels; ++p) t += tiles(N - p * nb, 3LL * k - p * nb);
+    const int outer = (N + kLuBlock - 1) / kLuBlock;
+    for (int p = 0; p < panels; ++p) t += tiles(N, kLuBlock);
+    for (int q = 0; q < outer; ++q) t += tiles(N - q * kLuBlock, 3LL * k - q * kLuBlock);
     for (int q = 0; q < back; ++q) t += tiles(static_cast<long long>(q) * kBackBlock, k);
-    const long long probs = 12 + panels + back;
+    const int ns = splitk_parts(n);
+    t += tiles(k, k) * 6LL * ns;                     // split-K partial products (S, P, Q, R, y)
+    const long long probs = 12 + panels + outer + back + 6LL * ns + 6;
     size_t b = static_cast<size_t>(t) * batch * sizeof(uint32_t) +
                static_cast<size_t>(probs) * batch * (sizeof(SimtProblem) + 16) + static_cast<size_t>(probs) * 2 * kAlign;
     return align_up(b + 4096, kAlign);
 }
 
-// Appends one grouped SIMT GEMM launch to the plan (f64_acc: fp64 accumulation).
-void add_gemm(Plan& plan, TableImage& img, const std::vector<SimtProblem>& probs, bool f64_acc = false) {
-    std::vector<uint32_t> tiles;
-    double flops = 0;
-    for (size_t p = 0; p < probs.size(); ++p) {
-        const SimtProblem& P = probs[p];
-        if (P.M <= 0 || P.N <= 0) continue;
-        const int mbs = (P.M + kSimtBM - 1) / kSimtBM, nbs = (P.N + kSimtBN - 1) / kSimtBN;
-        for (int nb = 0; nb < nbs; ++nb)
-            for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(static_cast<int>(p), mb, nb));
-        flops += 2.0 * P.M * P.N * P.K;
+// Appends grouped SIMT GEMM launches to the plan (f64_acc: fp64 accumulation), at most
+// kMaxTileProblems problems per launch.
+void add_gemm(Plan& plan, TableImage& img, const std::vector<SimtProblem>& all, bool f64_acc = false) {
+    for (size_t first = 0; first < all.size(); first += kMaxTileProblems) {
+        const size_t last = std::min(all.size(), first + static_cast<size_t>(kMaxTileProblems));
+        const std::vector<SimtProblem> probs(all.begin() + first, all.begin() + last);
+        std::vector<uint32_t> tiles;
+        double flops = 0;
+        for (size_t p = 0; p < probs.size(); ++p) {
+            const SimtProblem& P = probs[p];
+            if (P.M <= 0 || P.N <= 0) continue;
+            const int mbs = (P.M + kSimtBM - 1) / kSimtBM, nbs = (P.N + kSimtBN - 1) / kSimtBN;
+            for (int nb = 0; nb < nbs; ++nb)
+                for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(static_cast<int>(p), mb, nb));
+            flops += 2.0 * P.M * P.N * P.K;
+        }
+        if (tiles.empty()) continue;
+        const SimtProblem* dp = img.dev<SimtProblem>(img.add(probs.data(), probs.size() * sizeof(SimtProblem), kAlign));
+        const uint32_t* dt = img.dev<uint32_t>(img.add(tiles.data(), tiles.size() * sizeof(uint32_t), kAlign));
+        const int nt = static_cast<int>(tiles.size());
+        plan.steps.push_back({MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t s) {
+                                  return simt_gemm_launch(dp, dt, nt, s, f64_acc);
+                              }});
     }
-    if (tiles.empty()) return;
-    const SimtProblem* dp = img.dev<SimtProblem>(img.add(probs.data(), probs.size() * sizeof(SimtProblem), kAlign));
-    const uint32_t* dt = img.dev<uint32_t>(img.add(tiles.data(), tiles.size() * sizeof(uint32_t), kAlign));
-    const int nt = static_cast<int>(tiles.size());
-    plan.steps.push_back({MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t s) {
-                              return simt_gemm_launch(dp, dt, nt, s, f64_acc);
+}
+
+// The same products with the reduction dimension split into kSplitK chunks: every chunk's
+// fp32 partial goes to `part`, then one launch sums the partials in fp64 and applies
+// alpha, beta and the output type of each original problem.
+void add_gemm_splitk(Plan& plan, TableImage& img, const std::vector<SimtProblem>& probs, float* part) {
+    std::vector<SimtProblem> chunks;
+    std::vector<SplitKItem> items;
+    long long block0 = 0;
+    float* cur = part;
+    for (const SimtProblem& P : probs) {
+        const int ns = (P.K + kSplitK - 1) / kSplitK;
+        const long long mn = static_cast<long long>(P.M) * P.N;
+        for (int j = 0; j < ns; ++j) {
+            SimtProblem C = P;
+            const long long k0 = static_cast<long long>(j) * kSplitK;
+            C.A = static_cast<const uint8_t*>(P.A) + k0 * P.sak * (P.a_f64 ? 8 : 4);
+            C.B = static_cast<const uint8_t*>(P.B) + k0 * P.sbk * (P.b_f64 ? 8 : 4);
+            C.K = static_cast<int>(std::min<long long>(kSplitK, P.K - k0));
+            C.out = cur + j * mn;
+            C.out_f64 = 0;
+            C.ld_out = P.N;
+            C.E = nullptr;
+            C.alpha = 1.f;
+            C.beta = 0.f;
+            C.dscale = nullptr;
+            // vector loads stay legal: chunk offsets are multiples of 512 elements
+            chunks.push_back(C);
+        }
+        SplitKItem it;
+        std::memset(&it, 0, sizeof(it));
+        it.part = cur; it.out = P.out; it.E = P.E; it.ld_out = P.ld_out; it.ld_e = P.ld_e;
+        it.M = P.M; it.N = P.N; it.nsplit = ns; it.alpha = P.alpha; it.beta = P.beta;
+        it.out_f64 = P.out_f64; it.e_f64 = P.e_f64;
+        it.block0 = block0;
+        block0 += (mn + 255) / 256;
+        items.push_back(it);
+        cur += ns * mn;
+    }
+    add_gemm(plan, img, chunks, false);
+    const SplitKItem* di = img.dev<SplitKItem>(img.add(items.data(), items.size() * sizeof(SplitKItem), kAlign));
+    const int ni = static_cast<int>(items.size());
+    const long long nb = block0;
+    double bytes = 0;
+    for (const auto& it : items) bytes += 4.0 * it.nsplit * it.M * it.N + (it.out_f64 ? 8.0 : 4.0) * it.M * it.N;
+    plan.steps.push_back({MUON_KERNEL_MISC, bytes, [=](cudaStream_t s) {
+                              splitk_reduce_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(di, ni);
+                              return cudaGetLastError();
                           }});
 }
 
@@ -308,6 +461,7 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
     float* S = reinterpret_cast<float*>(ws + kHeaderBytes + L.S);
     double* Aug = reinterpret_cast<double*>(ws + kHeaderBytes + L.Aug);
     int* piv = reinterpret_cast<int*>(ws + kHeaderBytes + L.piv);
+    float* part = reinterpret_cast<float*>(ws + kHeaderBytes + L.part);
     const long long nk = static_cast<long long>(n) * k, kk = static_cast<long long>(k) * k;
     const int N = 2 * k, ncols = 3 * k;
     const long long ld = ncols, aug_stride = static_cast<long long>(N) * ncols;
@@ -322,9 +476,9 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
     auto Am = [&](int i, long long off) { return Mat{Ai(i) + off, ld, false, true}; };
 
     std::vector<SimtProblem> pr;
-    // S = W^T G (fp64 accumulation), then sym(S)
+    // S = W^T G (split-K), then sym(S)
     for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i, true), Gm(i), S + i * kk, k, false, nullptr, 0, false, k, k, n, 1.f, 0.f));
-    add_gemm(plan, img, pr, true); pr.clear();
+    add_gemm_splitk(plan, img, pr, part); pr.clear();
     plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * kk * B, [=](cudaStream_t s) {
         symmetrize_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(S, k, kk);
         return cudaGetLastError();
@@ -332,13 +486,13 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
     // V = G - W sym(S)
     for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Sm(i), V + i * nk, k, false, G + i * nk, k, false, n, k, k, -1.f, 1.f));
     add_gemm(plan, img, pr); pr.clear();
-    // fp64 blocks: [0,0] = c P = c W^T V, [0,k] = c Q = c W^T W, [k,0] = -c R = -c V^T V
+    // fp64 blocks (split-K sums): [0,0] = c P = c W^T V, [0,k] = c Q = c W^T W, [k,0] = -c R = -c V^T V
     for (int i = 0; i < B; ++i) {
         pr.push_back(gemm(Wm(i, true), Vm(i), Ai(i), ld, true, nullptr, 0, false, k, k, n, c, 0.f));
         pr.push_back(gemm(Wm(i, true), Wm(i), Ai(i) + k, ld, true, nullptr, 0, false, k, k, n, c, 0.f));
         pr.push_back(gemm(Vm(i, true), Vm(i), Ai(i) + k * ld, ld, true, nullptr, 0, false, k, k, n, -c, 0.f));
     }
-    add_gemm(plan, img, pr, true); pr.clear();
+    add_gemm_splitk(plan, img, pr, part); pr.clear();
     // [k,k] = -c P^T
     plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * kk * B, [=](cudaStream_t s) {
         aug_neg_transpose_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
@@ -354,40 +508,77 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
         aug_add_identity_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(Aug, N, ld, aug_stride);
         return cudaGetLastError();
     }});
-    // y = [W^T b; -V^T b] into the right-hand columns (fp64 accumulation)
+    // y = [W^T b; -V^T b] into the right-hand columns (split-K sums)
     for (int i = 0; i < B; ++i) {
         pr.push_back(gemm(Wm(i, true), bm(i), Ai(i) + N, ld, true, nullptr, 0, false, k, k, n, 1.f, 0.f));
         pr.push_back(gemm(Vm(i, true), bm(i), Ai(i) + k * ld + N, ld, true, nullptr, 0, false, k, k, n, -1.f, 0.f));
     }
-    add_gemm(plan, img, pr, true); pr.clear();
-    // Gaussian elimination with partial pivoting on [C | y], fp64
+    add_gemm_splitk(plan, img, pr, part); pr.clear();
+    // Gaussian elimination with partial pivoting on [C | y], fp64, two levels: 128-column
+    // block columns factorised with nb-wide panels (updates confined to the block column),
+    // then one row-swap + unit-lower solve over the trailing columns and one K = 128
+    // trailing update per block column.
     const int nb = lu_panel_width(N);
-    for (int j0 = 0; j0 < N; j0 += nb) {
-        const int w = std::min(nb, N - j0);
-        const size_t smem = static_cast<size_t>(N - j0) * w * sizeof(double);
-        const double lu_flops = 2.0 * (N - j0) * w * w * B;
-        plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
-            static bool attr = false;
-            if (!attr) {
-                cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
-                attr = true;
-            }
-            lu_panel_kernel<<<B, 1024, smem, s>>>(Aug, ld, aug_stride, N, j0, w, piv, N, d_status);
-            return cudaGetLastError();
-        }});
-        const int right = ncols - (j0 + w);
-        if (right > 0) {
-            plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right * B, [=](cudaStream_t s) {
-                lu_swap_trsm_kernel<<<dim3((right + 127) / 128, B), 128, static_cast<size_t>(w) * w * sizeof(double), s>>>(
-                    Aug, ld, aug_stride, j0, w, ncols, piv, N);
+    for (int J0 = 0; J0 < N; J0 += kLuBlock) {
+        const int JB = std::min(kLuBlock, N - J0);
+        for (int j0 = J0; j0 < J0 + JB; j0 += nb) {
+            const int w = std::min(nb, J0 + JB - j0);
+            const size_t smem = static_cast<size_t>(N - j0) * w * sizeof(double);
+            const double lu_flops = 2.0 * (N - j0) * w * w * B;
+            plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
+                static bool attr = false;
+                if (!attr) {
+                    cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
+                    attr = true;
+                }
+                lu_panel_kernel<<<B, 1024, smem, s>>>(Aug, ld, aug_stride, N, j0, w, piv, N, d_status);
                 return cudaGetLastError();
             }});
-            if (N - j0 - w > 0) {
+            if (j0 > J0) {
+                const int left = j0 - J0;
+                plan.steps.push_back({MUON_KERNEL_LU, 0.0, [=](cudaStream_t s) {
+                    lu_swap_cols_kernel<<<dim3((left + 127) / 128, B), 128, 0, s>>>(Aug, ld, aug_stride, J0, j0, j0, w,
+                                                                                    piv, N);
+                    return cudaGetLastError();
+                }});
+            }
+            const int right_in = J0 + JB - (j0 + w);
+            if (right_in > 0) {
+                const int block_end = J0 + JB;
+                plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right_in * B, [=](cudaStream_t s) {
+                    lu_swap_trsm_kernel<<<dim3((right_in + 127) / 128, B), 128, static_cast<size_t>(w) * w * sizeof(double), s>>>(
+                        Aug, ld, aug_stride, j0, w, block_end, piv, N);
+                    return cudaGetLastError();
+                }});
                 for (int i = 0; i < B; ++i) {
                     double* base = Ai(i);
                     pr.push_back(gemm(Mat{base + (j0 + w) * ld + j0, ld, false, true}, Mat{base + j0 * ld + j0 + w, ld, false, true},
                                       base + (j0 + w) * ld + j0 + w, ld, true, base + (j0 + w) * ld + j0 + w, ld, true,
-                                      N - j0 - w, right, w, -1.f, 1.f));
+                                      N - j0 - w, right_in, w, -1.f, 1.f));
+                }
+                add_gemm(plan, img, pr, true); pr.clear();
+            }
+        }
+        const int right = ncols - (J0 + JB);
+        if (right > 0) {
+            const int c_lo = J0 + JB;
+            plan.steps.push_back({MUON_KERNEL_LU, 1.0 * JB * JB * right * B, [=](cudaStream_t s) {
+                static bool attr = false;
+                if (!attr) {
+                    cudaFuncSetAttribute(lu_block_swap_trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kLuBlock * kLuBlock * static_cast<int>(sizeof(double)));
+                    attr = true;
+                }
+                lu_block_swap_trsm_kernel<<<dim3((right + 127) / 128, B), 128, static_cast<size_t>(JB) * JB * sizeof(double), s>>>(
+                    Aug, ld, aug_stride, J0, JB, c_lo, ncols, piv, N);
+                return cudaGetLastError();
+            }});
+            if (N - J0 - JB > 0) {
+                for (int i = 0; i < B; ++i) {
+                    double* base = Ai(i);
+                    pr.push_back(gemm(Mat{base + (J0 + JB) * ld + J0, ld, false, true}, Mat{base + J0 * ld + J0 + JB, ld, false, true},
+                                      base + (J0 + JB) * ld + J0 + JB, ld, true, base + (J0 + JB) * ld + J0 + JB, ld, true,
+                                      N - J0 - JB, right, JB, -1.f, 1.f));
                 }
                 add_gemm(plan, img, pr, true); pr.clear();
             }
