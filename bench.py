@@ -151,7 +151,7 @@ def _time_ms(fn, warmup, steps):
     return e0.elapsed_time(e1) / steps
 
 
-def secondary_measurements():
+def secondary_measurements(only=None):
     """The other parameter sets of the method, each timed on the device (CUDA events,
     warm-up first): a 64 x 1024^2 low-rank batch through ns_orthogonalize under the fixed and
     the hybrid schedule, the GPT-2-small set's full step, the 16 x 4096 x 1024 Stiefel step
@@ -160,7 +160,24 @@ def secondary_measurements():
     from matrix_orthogonalising_optimizer_02_b200 import binding as mb
     from matrix_orthogonalising_optimizer_02_b200 import workloads
     out = {}
-    # low-rank batch
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1003)
+    if only in (None, "lowrank"):
+        out.update(_lowrank())
+    if only in (None, "gpt2"):
+        out.update(_gpt2(gen))
+    if only in (None, "stiefel"):
+        out.update(_stiefel(gen))
+    if only in (None, "single"):
+        out.update(_single())
+    return out
+
+
+def _lowrank():
+    import torch
+    from matrix_orthogonalising_optimizer_02_b200 import binding as mb
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    out = {}
     X = torch.tensor(workloads.low_rank_plus_noise(batch=64, n=1024)).to(torch.bfloat16).cuda()
     Y = torch.empty_like(X)
     for name, sch, iters in [("lowrank64_kj5_split2", mb.Schedule.fixed(5, n_split_iters=2), 5),
@@ -170,10 +187,14 @@ def secondary_measurements():
         fl = 64 * iters * 4.0 * 1024 ** 3
         out[name] = {"ms": ms, "algorithmic_tflops": fl / (ms * 1e-3) / 1e12}
         del ws
-    del X, Y
-    # GPT-2-small set
-    gen = torch.Generator(device="cuda")
-    gen.manual_seed(1003)
+    return out
+
+
+def _gpt2(gen):
+    import torch
+    from matrix_orthogonalising_optimizer_02_b200 import binding as mb
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    out = {}
     mats = []
     for (rows, cols) in workloads.gpt2_small_shapes(12):
         mats.append(mb.Matrix(torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda").normal_(0, 0.02, generator=gen),
@@ -184,8 +205,14 @@ def secondary_measurements():
     ms = _time_ms(lambda: mb.muon_step_batched(mats, hp, ws), 3, 10)
     fl = sum(ns_flops_algorithmic(r, c) for r, c in workloads.gpt2_small_shapes(12))
     out["gpt2_small_step"] = {"ms": ms, "ns_algorithmic_tflops": fl / (ms * 1e-3) / 1e12}
-    del mats, ws
-    # Stiefel step
+    return out
+
+
+def _stiefel(gen):
+    import torch
+    from matrix_orthogonalising_optimizer_02_b200 import binding as mb
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    out = {}
     W = torch.tensor(workloads.stiefel_problem(batch=16, n=4096, k=1024), dtype=torch.float32, device="cuda")
     G = torch.empty_like(W).normal_(0, 1.0, generator=gen)
     ws = mb.workspace(mb.stiefel_workspace_size(16, 4096, 1024))
@@ -194,14 +221,20 @@ def secondary_measurements():
     mb.stiefel_cayley_step(W, G, 1e-2, ws)
     torch.cuda.synchronize()
     mb.timing_enable(False)
-    kinds = {k: mb.timing_read(k) for k in ("simt_gemm", "lu", "misc")}
-    work = kinds["simt_gemm"][2] + kinds["lu"][2]
+    kinds = {k: mb.timing_read(k) for k in ("tc_f32", "simt_gemm", "lu", "misc")}
+    work = kinds["tc_f32"][2] + kinds["simt_gemm"][2] + kinds["lu"][2]
     ms = _time_ms(lambda: mb.stiefel_cayley_step(W, G, 1e-2, ws), 1, 3)
     out["stiefel_16x4096x1024_step"] = {"ms": ms, "fma_tflops": work / (ms * 1e-3) / 1e12,
                                         "kernel_ms": {k: v[0] for k, v in kinds.items()},
-                                        "simt_gemm_tflops": kinds["simt_gemm"][2] / (kinds["simt_gemm"][0] * 1e-3) / 1e12}
-    del W, G, ws
-    # single fp32 matrix
+                                        "tc_f32_tflops": kinds["tc_f32"][2] / max(kinds["tc_f32"][0] * 1e-3, 1e-12) / 1e12}
+    return out
+
+
+def _single():
+    import torch
+    from matrix_orthogonalising_optimizer_02_b200 import binding as mb
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    out = {}
     Wn, Gn, Mn = workloads.single_fp32()
     one = [mb.Matrix(torch.tensor(Wn).cuda(), torch.tensor(Gn).cuda(), torch.tensor(Mn).cuda())]
     hp1 = mb.hyper(lr=0.02, beta=0.95, weight_decay=0.0, schedule=mb.Schedule.fixed(5, fp32_mode=True))
@@ -243,6 +276,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-secondary", action="store_true", help="skip the other parameter sets")
+    ap.add_argument("--case", default=None, choices=["lowrank", "gpt2", "stiefel", "single"],
+                    help="time only one of the other parameter sets (for profiling); prints its figures")
     ap.add_argument("--layers", type=int, default=32,
                     help="Llama-7B layers in the set (32 = the full set; 1 = a profiling-sized case)")
     args = ap.parse_args()
@@ -255,6 +290,9 @@ def main():
         run_reference(args, rank, world)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"
+    if args.case is not None:
+        print(json.dumps(secondary_measurements(only=args.case)), flush=True)
+        return
 
     import datetime
     import torch

@@ -198,8 +198,9 @@ typedef enum {
     MUON_KERNEL_UPDATE = 3,       /* scale + decoupled weight decay + update              */
     MUON_KERNEL_SIMT_GEMM = 4,    /* fp32 FMA GEMMs (fp32 NS mode, Stiefel)               */
     MUON_KERNEL_LU = 5,           /* 2k x 2k LU and triangular solves                     */
-    MUON_KERNEL_MISC = 6,         /* casts, copies, block assembly                        */
-    MUON_KERNEL_KINDS = 7
+    MUON_KERNEL_MISC = 6,         /* casts, copies, block assembly, plane splits          */
+    MUON_KERNEL_TC_F32 = 7,       /* tcgen05 fp32 products from three bf16 planes (Stiefel) */
+    MUON_KERNEL_KINDS = 8
 } muon_kernel_kind;
 MUON_API muon_status muon_timing_enable(int enable);
 MUON_API muon_status muon_timing_reset(void);

@@ -22,7 +22,8 @@ MUON_ERR_WORKSPACE_TOO_SMALL, MUON_ERR_CUDA, MUON_ERR_NONFINITE, MUON_ERR_DEVICE
 MUON_BF16, MUON_F32 = 0, 1
 SCALE_MODES = {"moonlight": 0, "kellerjordan": 1, "mup": 2, "naive": 3}
 MUON_MAX_NS_ITERS = 32
-KERNEL_KINDS = {"momentum": 0, "scale": 1, "ns_gemm": 2, "update": 3, "simt_gemm": 4, "lu": 5, "misc": 6}
+KERNEL_KINDS = {"momentum": 0, "scale": 1, "ns_gemm": 2, "update": 3, "simt_gemm": 4, "lu": 5, "misc": 6,
+                "tc_f32": 7}
 
 #: Exported entry points, as declared in include/muon_b200.h.
 EXPORTED = (

@@ -16,26 +16,51 @@ constexpr unsigned kDevErrNonfinite = 2u;
 // One problem of a grouped launch: out = f * (alpha * (A_op x B_op) + beta * E), f = 1 or
 // (*dscale)^scale_pow, on bf16 operands with fp32 accumulation in TMEM.  A_op is M x K,
 // B_op is K x N; each is read through TMA tensor maps, K-major (contiguous along K) or
-// MN-major (contiguous along M resp. N).  A second ("lo") plane of an operand adds the
-// split-bf16 products hi*lo and lo*hi.  With kSym the output is symmetric: only tiles that
-// reach the upper triangle are computed, and their elements above the diagonal are also
-// stored mirrored.
+// MN-major (contiguous along M resp. N).  An operand may come as up to three bf16 planes
+// (value = plane0 + plane1 + plane2); the K loop runs over a list of plane pairs
+// ("segments"), e.g. (0,0),(0,1),(1,0) for split-bf16, or the six pairs with indices
+// summing to <= 2 for an fp32 operand split into three planes.  K starts at k_begin
+// (split-K chunks).  The output is bf16 (plane 0 = value, optional plane 1 = remainder)
+// or fp32; E is bf16 (one or two planes) or fp32.  With kProbSym the output is
+// symmetric: only tiles that reach the upper triangle are computed, and their elements
+// above the diagonal are also stored mirrored.
 constexpr uint32_t kProbAMn = 1u;
 constexpr uint32_t kProbBMn = 2u;
 constexpr uint32_t kProbSym = 4u;
+constexpr uint32_t kProbOutF32 = 8u;
+constexpr uint32_t kProbEF32 = 16u;
+constexpr int kTcMaxPlanes = 3, kTcMaxSegments = 8;
 
 struct alignas(16) TcProblem {
-    const CUtensorMap* tmA[2];
-    const CUtensorMap* tmB[2];
-    const __nv_bfloat16* E[2];
-    __nv_bfloat16* out[2];
+    const CUtensorMap* tmA[kTcMaxPlanes];
+    const CUtensorMap* tmB[kTcMaxPlanes];
+    const void* E[2];
+    void* out[2];
     const float* dscale;
     int M, N, K;
+    int k_begin;
     int ld;            // row pitch (elements) of out and E
     float alpha, beta;
     int scale_pow;
     uint32_t flags;
+    int nseg;
+    uint32_t segs;     // segment s: A plane = (segs >> 4s) & 3, B plane = (segs >> (4s + 2)) & 3
 };
+
+// Segment list of plane pairs (pa, pb) with pa < na, pb < nb and pa + pb <= max_order,
+// ordered by pa + pb (largest terms first).
+inline void tc_set_segments(TcProblem& P, int na, int nb, int max_order) {
+    P.nseg = 0;
+    P.segs = 0;
+    for (int o = 0; o <= max_order; ++o)
+        for (int pa = 0; pa <= o; ++pa) {
+            const int pb = o - pa;
+            if (pa < na && pb < nb && P.nseg < kTcMaxSegments) {
+                P.segs |= static_cast<uint32_t>(pa | (pb << 2)) << (4 * P.nseg);
+                ++P.nseg;
+            }
+        }
+}
 
 constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64, kTcStages = 6;   // pair (2-CTA) tile
 constexpr int kTcThreads = 384;            // 4 role warps + 8 epilogue warps
@@ -67,6 +92,7 @@ struct alignas(16) SimtProblem {
     int scale_pow;
     int vec_a, vec_b;  // 16-byte vector loads allowed along the contiguous dimension
     int a_f64, b_f64, e_f64, out_f64;
+    int sym;           // symmetric output: only tiles with n-block >= m-block; mirrored stores
 };
 constexpr int kSimtBM = 128, kSimtBN = 128, kSimtBK = 8, kSimtThreads = 256;
 cudaError_t simt_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream,

@@ -109,29 +109,6 @@ size_t ns_tables_bound(const std::vector<std::pair<int, int>>& shapes, const muo
     return b;
 }
 
-// ---------------------------------------------------------------- tensor-map pool
-struct TmapPool {
-    TableImage& img;
-    struct Entry {
-        const void* base;
-        int rows, cols, box;
-        size_t off;
-    };
-    std::vector<Entry> entries;
-    bool failed = false;
-    explicit TmapPool(TableImage& i) : img(i) {}
-    const CUtensorMap* get(const void* base, int rows, int cols, int box) {
-        if (base == nullptr) return nullptr;
-        for (auto& e : entries)
-            if (e.base == base && e.rows == rows && e.cols == cols && e.box == box) return img.dev<CUtensorMap>(e.off);
-        CUtensorMap tm;
-        if (!encode_bf16_tmap(&tm, base, rows, cols, box)) failed = true;
-        const size_t off = img.add(&tm, sizeof(tm), 128);
-        entries.push_back({base, rows, cols, box, off});
-        return img.dev<CUtensorMap>(off);
-    }
-};
-
 // TMA boxes: 64 bf16 (128 B) of the contiguous dimension x 128 rows (K-major operand half
 // of a pair tile), or 64 x 64 (one MN-major chunk).
 constexpr int kBoxK = kTcBM / 2, kBoxMN = 64;
@@ -188,8 +165,8 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                     P.tmA[1] = pool.get(a1, r, r, kBoxK);
                     P.tmB[0] = P.tmA[0];
                     P.tmB[1] = P.tmA[1];
-                    P.E[0] = static_cast<const __nv_bfloat16*>(m.A[0]);
-                    P.E[1] = static_cast<const __nv_bfloat16*>(a1);
+                    P.E[0] = m.A[0];
+                    P.E[1] = a1;
                     P.out[0] = static_cast<__nv_bfloat16*>(m.B[0]);
                     P.out[1] = split ? static_cast<__nv_bfloat16*>(m.B[1]) : nullptr;
                     P.M = r; P.N = r; P.K = r; P.ld = r;
@@ -211,8 +188,8 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                         P.tmB[1] = pool.get(b1, r, r, kBoxK);
                         P.flags = 0;
                     }
-                    P.E[0] = static_cast<const __nv_bfloat16*>(xin0);
-                    P.E[1] = static_cast<const __nv_bfloat16*>(xin1);
+                    P.E[0] = xin0;
+                    P.E[1] = xin1;
                     void* out0 = (last && m.final_out) ? m.final_out : m.X[nxt][0];
                     P.out[0] = static_cast<__nv_bfloat16*>(out0);
                     P.out[1] = split ? static_cast<__nv_bfloat16*>(m.X[nxt][1]) : nullptr;
@@ -223,6 +200,8 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                     flops += 2.0 * r * r * s;
                     if (last) final_x[order[pi]] = out0;
                 }
+                // split-bf16: hi*hi + hi*lo + lo*hi over the planes present
+                tc_set_segments(P, P.tmA[1] ? 2 : 1, P.tmB[1] ? 2 : 1, 1);
                 probs.push_back(P);
                 const int p = static_cast<int>(probs.size()) - 1;
                 if (stage < 2) {

@@ -90,6 +90,29 @@ muon_status run_plan(const std::vector<uint8_t>& key, void* workspace, size_t ta
 // x box_rows rows, 128-byte swizzle, zero fill out of bounds.
 bool encode_bf16_tmap(CUtensorMap* out, const void* base, int rows, int cols, int box_rows);
 
+// Tensor maps of one plan, deduplicated by (base, shape, box), stored in the table image.
+struct TmapPool {
+    TableImage& img;
+    struct Entry {
+        const void* base;
+        int rows, cols, box;
+        size_t off;
+    };
+    std::vector<Entry> entries;
+    bool failed = false;
+    explicit TmapPool(TableImage& i) : img(i) {}
+    const CUtensorMap* get(const void* base, int rows, int cols, int box) {
+        if (base == nullptr) return nullptr;
+        for (auto& e : entries)
+            if (e.base == base && e.rows == rows && e.cols == cols && e.box == box) return img.dev<CUtensorMap>(e.off);
+        CUtensorMap tm;
+        if (!encode_bf16_tmap(&tm, base, rows, cols, box)) failed = true;
+        const size_t off = img.add(&tm, sizeof(tm), 128);
+        entries.push_back({base, rows, cols, box, off});
+        return img.dev<CUtensorMap>(off);
+    }
+};
+
 int device_sm_count();
 muon_status from_cuda(cudaError_t e);
 

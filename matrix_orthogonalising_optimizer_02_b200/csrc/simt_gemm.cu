@@ -13,24 +13,29 @@ namespace {
 constexpr int BM = kSimtBM, BN = kSimtBN, BK = kSimtBK;
 constexpr int PAD = 4;
 
-__device__ __forceinline__ double ld1(const void* base, long long off, int f64) {
-    return f64 ? __ldg(static_cast<const double*>(base) + off) : static_cast<double>(__ldg(static_cast<const float*>(base) + off));
+template <class T>
+__device__ __forceinline__ T ld1(const void* base, long long off, int f64) {
+    return f64 ? static_cast<T>(__ldg(static_cast<const double*>(base) + off))
+               : static_cast<T>(__ldg(static_cast<const float*>(base) + off));
 }
-__device__ __forceinline__ void ld4(const void* base, long long off, int f64, double (&r)[4]) {
+template <class T>
+__device__ __forceinline__ void ld4(const void* base, long long off, int f64, T (&r)[4]) {
     if (f64) {
         const double2 a = __ldg(reinterpret_cast<const double2*>(static_cast<const double*>(base) + off));
         const double2 b = __ldg(reinterpret_cast<const double2*>(static_cast<const double*>(base) + off) + 1);
-        r[0] = a.x; r[1] = a.y; r[2] = b.x; r[3] = b.y;
+        r[0] = static_cast<T>(a.x); r[1] = static_cast<T>(a.y); r[2] = static_cast<T>(b.x); r[3] = static_cast<T>(b.y);
     } else {
         const float4 v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + off));
-        r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+        r[0] = static_cast<T>(v.x); r[1] = static_cast<T>(v.y); r[2] = static_cast<T>(v.z); r[3] = static_cast<T>(v.w);
     }
 }
 
 // Thread -> element mapping of a tile load.  If the operand is contiguous along K the
 // 256 threads cover 128 rows x 2 quads of K; otherwise 8 K-rows x 32 quads of M (or N).
+// Values arrive in the accumulator type T (fp64 sources are rounded when T is float).
+template <class T>
 __device__ __forceinline__ void load_tile(const void* __restrict__ base, int f64, long long s_mn, long long s_k,
-                                          int mn0, int k0, int MN, int K, int vec, int tid, double (&r)[4]) {
+                                          int mn0, int k0, int MN, int K, int vec, int tid, T (&r)[4]) {
     const bool k_contig = (s_k == 1);
     int mn, k;
     if (k_contig) {
@@ -46,20 +51,20 @@ __device__ __forceinline__ void load_tile(const void* __restrict__ base, int f64
             ld4(base, gm * s_mn + gk, f64, r);
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) r[i] = (gm < MN && gk + i < K) ? ld1(base, gm * s_mn + (gk + i) * s_k, f64) : 0.0;
+            for (int i = 0; i < 4; ++i) r[i] = (gm < MN && gk + i < K) ? ld1<T>(base, gm * s_mn + (gk + i) * s_k, f64) : T(0);
         }
     } else {
         if (vec && gk < K && gm + 3 < MN) {
             ld4(base, gm * s_mn + gk * s_k, f64, r);
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) r[i] = (gk < K && gm + i < MN) ? ld1(base, (gm + i) * s_mn + gk * s_k, f64) : 0.0;
+            for (int i = 0; i < 4; ++i) r[i] = (gk < K && gm + i < MN) ? ld1<T>(base, (gm + i) * s_mn + gk * s_k, f64) : T(0);
         }
     }
 }
 
 template <class Acc>
-__device__ __forceinline__ void store_tile(Acc (*s)[BM + PAD], bool k_contig, int tid, const double (&r)[4]) {
+__device__ __forceinline__ void store_tile(Acc (*s)[BM + PAD], bool k_contig, int tid, const Acc (&r)[4]) {
     if (k_contig) {
         const int mn = tid >> 1, k = (tid & 1) * 4;
 #pragma unroll
@@ -67,8 +72,7 @@ __device__ __forceinline__ void store_tile(Acc (*s)[BM + PAD], bool k_contig, in
     } else {
         const int k = tid >> 5, mn = (tid & 31) * 4;
         if constexpr (sizeof(Acc) == sizeof(float)) {
-            *reinterpret_cast<float4*>(&s[k][mn]) = make_float4(static_cast<float>(r[0]), static_cast<float>(r[1]),
-                                                                static_cast<float>(r[2]), static_cast<float>(r[3]));
+            *reinterpret_cast<float4*>(&s[k][mn]) = make_float4(r[0], r[1], r[2], r[3]);
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i) s[k][mn + i] = static_cast<Acc>(r[i]);
@@ -90,8 +94,9 @@ __device__ __forceinline__ void load4(const float* p, float (&v)[8], int o) {
     v[o] = q.x; v[o + 1] = q.y; v[o + 2] = q.z; v[o + 3] = q.w;
 }
 
+// fp32: two CTAs (16 warps) per SM; fp64: one (its 8 x 8 fp64 block needs the registers).
 template <class Acc>
-__global__ void __launch_bounds__(kSimtThreads)
+__global__ void __launch_bounds__(kSimtThreads, sizeof(Acc) == sizeof(float) ? 2 : 1)
 simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restrict__ tiles, int num_tiles) {
     __shared__ __align__(16) Acc As[2][BK][BM + PAD];
     __shared__ __align__(16) Acc Bs[2][BK][BN + PAD];
@@ -112,7 +117,7 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[i][j] = Acc(0);
 
-        double ra[4], rb[4];
+        Acc ra[4], rb[4];
         // A(m, k) = A[m*sam + k*sak]; B(k, n) = B[k*sbk + n*sbn] -> as an (n, k) operand.
         load_tile(P.A, P.a_f64, P.sam, P.sak, m0, 0, P.M, P.K, P.vec_a, tid, ra);
         load_tile(P.B, P.b_f64, P.sbn, P.sbk, n0, 0, P.N, P.K, P.vec_b, tid, rb);
@@ -162,6 +167,7 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
             for (int j = 0; j < 8; ++j) {
                 const int n = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
                 if (n >= P.N) continue;
+                if (P.sym && n < m) continue;   // written by the mirror of (n, m)
                 Acc v = static_cast<Acc>(alpha) * acc[i][j];
                 if (beta != 0.f) {
                     const long long eo = static_cast<long long>(m) * P.ld_e + n;
@@ -170,8 +176,14 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
                     v = fma(static_cast<Acc>(beta), e, v);
                 }
                 const long long oo = static_cast<long long>(m) * P.ld_out + n;
-                if (P.out_f64) static_cast<double*>(P.out)[oo] = static_cast<double>(v);
-                else static_cast<float*>(P.out)[oo] = static_cast<float>(v);
+                const long long om = static_cast<long long>(n) * P.ld_out + m;
+                if (P.out_f64) {
+                    static_cast<double*>(P.out)[oo] = static_cast<double>(v);
+                    if (P.sym && n > m) static_cast<double*>(P.out)[om] = static_cast<double>(v);
+                } else {
+                    static_cast<float*>(P.out)[oo] = static_cast<float>(v);
+                    if (P.sym && n > m) static_cast<float*>(P.out)[om] = static_cast<float>(v);
+                }
             }
         }
     }

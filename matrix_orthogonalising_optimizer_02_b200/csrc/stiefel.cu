@@ -127,6 +127,39 @@ __global__ void splitk_reduce_kernel(const SplitKItem* __restrict__ items, int c
     else static_cast<float*>(it.out)[oo] = static_cast<float>(v);
 }
 
+// Exact three-way bf16 split of an fp32 value (fp64 sources are first rounded to fp32):
+// x = hi + mid + lo with hi = bf16(x), mid = bf16(x - hi), lo = x - hi - mid (8 bits each).
+struct Split3Item {
+    const void* src;
+    __nv_bfloat16* dst;   // 3 planes of rows x cols, contiguous
+    long long ld;
+    long long block0;
+    int rows, cols;
+    int src_f64;
+};
+__global__ void split3_kernel(const Split3Item* __restrict__ items, int count) {
+    const long long b = blockIdx.x;
+    int lo = 0, hi = count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (items[mid].block0 <= b) lo = mid; else hi = mid - 1;
+    }
+    const Split3Item& it = items[lo];
+    const long long n = static_cast<long long>(it.rows) * it.cols;
+    const long long e = (b - it.block0) * blockDim.x + threadIdx.x;
+    if (e >= n) return;
+    const long long r = e / it.cols, c = e % it.cols;
+    const float x = it.src_f64 ? static_cast<float>(static_cast<const double*>(it.src)[r * it.ld + c])
+                               : static_cast<const float*>(it.src)[r * it.ld + c];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    it.dst[e] = h;
+    it.dst[n + e] = m;
+    it.dst[2 * n + e] = __float2bfloat16_rn(r2);
+}
+
 // Panel factorisation (partial pivoting) of rows j0..N-1, columns j0..j0+nb-1, held in
 // shared memory.  Records the pivot row of each column in piv (absolute row indices).
 __global__ void __launch_bounds__(1024)
@@ -309,8 +342,16 @@ int lu_panel_width(int N) {
 }
 
 struct StiefelLayout {
-    size_t V, b, S, Aug, piv, cm, part, table_offset, data_bytes;
+    size_t V, b, S, Aug, piv, cm, part, planes, table_offset, data_bytes;
+    bool tc;
 };
+
+// The tensor-core plan needs 16-byte bf16 row pitches for TMA.
+bool stiefel_tc_ok(int n, int k) { return n % 8 == 0 && k % 8 == 0; }
+// bf16 planes per matrix: W, G (n x k) and S (k x k), 3 planes each.
+size_t stiefel_plane_elems(int n, int k) {
+    return 3 * (2 * static_cast<size_t>(n) * k + static_cast<size_t>(k) * k);
+}
 
 // Split-K for the reductions over n: chunks of kSplitK rows summed in fp32, chunk partial
 // sums added in fp64 in a fixed order.
@@ -328,6 +369,8 @@ StiefelLayout stiefel_layout(int batch, int n, int k) {
     L.cm = ar.take(static_cast<size_t>(k) * sizeof(double) * batch);
     // largest split-K group: the three k x k blocks P, Q, R of every matrix
     L.part = ar.take(static_cast<size_t>(3) * batch * splitk_parts(n) * k * k * sizeof(float));
+    L.tc = stiefel_tc_ok(n, k);
+    L.planes = L.tc ? ar.take(stiefel_plane_elems(n, k) * sizeof(__nv_bfloat16) * batch) : 0;
     L.data_bytes = align_up(ar.used, kAlign);
     L.table_offset = kHeaderBytes + L.data_bytes;
     return L;
@@ -347,8 +390,13 @@ size_t stiefel_tables_bound(int batch, int n, int k) {
     const int ns = splitk_parts(n);
     t += tiles(k, k) * 6LL * ns;                     // split-K partial products (S, P, Q, R, y)
     const long long probs = 12 + panels + outer + back + 6LL * ns + 6;
-    size_t b = static_cast<size_t>(t) * batch * sizeof(uint32_t) +
-               static_cast<size_t>(probs) * batch * (sizeof(SimtProblem) + 16) + static_cast<size_t>(probs) * 2 * kAlign;
+    // tensor-core products (S split-K chunks, V): tiles, tensor maps of 3 plane sets x 3
+    // planes x 2 box shapes, split items
+    t += (tiles(k, k) * ns + tiles(n, k)) * 2LL;
+    const size_t tmaps = static_cast<size_t>(batch) * 3 * 3 * 2 * (sizeof(CUtensorMap) + 128);
+    const size_t prob_bytes = std::max(sizeof(SimtProblem), sizeof(TcProblem)) + 16;
+    size_t b = static_cast<size_t>(t) * batch * sizeof(uint32_t) + static_cast<size_t>(probs) * batch * prob_bytes +
+               static_cast<size_t>(probs) * 2 * kAlign + tmaps + static_cast<size_t>(batch) * 16 * 64 + 64 * kAlign;
     return align_up(b + 4096, kAlign);
 }
 
@@ -365,8 +413,9 @@ void add_gemm(Plan& plan, TableImage& img, const std::vector<SimtProblem>& all, 
             if (P.M <= 0 || P.N <= 0) continue;
             const int mbs = (P.M + kSimtBM - 1) / kSimtBM, nbs = (P.N + kSimtBN - 1) / kSimtBN;
             for (int nb = 0; nb < nbs; ++nb)
-                for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(static_cast<int>(p), mb, nb));
-            flops += 2.0 * P.M * P.N * P.K;
+                for (int mb = 0; mb < mbs; ++mb)
+                    if (!P.sym || nb >= mb) tiles.push_back(tile_code(static_cast<int>(p), mb, nb));
+            flops += (P.sym ? 1.0 : 2.0) * P.M * P.N * P.K;
         }
         if (tiles.empty()) continue;
         const SimtProblem* dp = img.dev<SimtProblem>(img.add(probs.data(), probs.size() * sizeof(SimtProblem), kAlign));
@@ -451,69 +500,12 @@ SimtProblem gemm(Mat A, Mat B, void* out, long long ldo, bool o64, const void* E
     return P;
 }
 
-// Appends the projection + Woodbury-Cayley launches for W (batch x n x k) with direction
-// source G (may be the workspace V buffer itself: V = G - W sym(W^T G) is then formed in
-// place, each element read and written by one thread).
-muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, uint8_t* ws, unsigned* d_status,
-                          float* W, const float* G, int batch, int n, int k, float lr, size_t ws_bytes) {
-    float* V = reinterpret_cast<float*>(ws + kHeaderBytes + L.V);
-    float* bb = reinterpret_cast<float*>(ws + kHeaderBytes + L.b);
-    float* S = reinterpret_cast<float*>(ws + kHeaderBytes + L.S);
-    double* Aug = reinterpret_cast<double*>(ws + kHeaderBytes + L.Aug);
-    int* piv = reinterpret_cast<int*>(ws + kHeaderBytes + L.piv);
-    float* part = reinterpret_cast<float*>(ws + kHeaderBytes + L.part);
-    const long long nk = static_cast<long long>(n) * k, kk = static_cast<long long>(k) * k;
-    const int N = 2 * k, ncols = 3 * k;
-    const long long ld = ncols, aug_stride = static_cast<long long>(N) * ncols;
-    const float c = 0.5f * lr;
-    const int B = batch;
-    auto Wm = [&](int i, bool t = false) { return Mat{W + i * nk, k, t, false}; };
-    auto Gm = [&](int i) { return Mat{G + i * nk, k, false, false}; };
-    auto Vm = [&](int i, bool t = false) { return Mat{V + i * nk, k, t, false}; };
-    auto bm = [&](int i) { return Mat{bb + i * nk, k, false, false}; };
-    auto Sm = [&](int i) { return Mat{S + i * kk, k, false, false}; };
+// Gaussian elimination with partial pivoting on the augmented fp64 systems [C | y]
+// (N x ncols, row pitch ld, batch B), then back substitution: z overwrites y.
+void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int ncols, int k, int B, long long ld,
+                  long long aug_stride, unsigned* d_status) {
     auto Ai = [&](int i) { return Aug + i * aug_stride; };
-    auto Am = [&](int i, long long off) { return Mat{Ai(i) + off, ld, false, true}; };
-
     std::vector<SimtProblem> pr;
-    // S = W^T G (split-K), then sym(S)
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i, true), Gm(i), S + i * kk, k, false, nullptr, 0, false, k, k, n, 1.f, 0.f));
-    add_gemm_splitk(plan, img, pr, part); pr.clear();
-    plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * kk * B, [=](cudaStream_t s) {
-        symmetrize_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(S, k, kk);
-        return cudaGetLastError();
-    }});
-    // V = G - W sym(S)
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Sm(i), V + i * nk, k, false, G + i * nk, k, false, n, k, k, -1.f, 1.f));
-    add_gemm(plan, img, pr); pr.clear();
-    // fp64 blocks (split-K sums): [0,0] = c P = c W^T V, [0,k] = c Q = c W^T W, [k,0] = -c R = -c V^T V
-    for (int i = 0; i < B; ++i) {
-        pr.push_back(gemm(Wm(i, true), Vm(i), Ai(i), ld, true, nullptr, 0, false, k, k, n, c, 0.f));
-        pr.push_back(gemm(Wm(i, true), Wm(i), Ai(i) + k, ld, true, nullptr, 0, false, k, k, n, c, 0.f));
-        pr.push_back(gemm(Vm(i, true), Vm(i), Ai(i) + k * ld, ld, true, nullptr, 0, false, k, k, n, -c, 0.f));
-    }
-    add_gemm_splitk(plan, img, pr, part); pr.clear();
-    // [k,k] = -c P^T
-    plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * kk * B, [=](cudaStream_t s) {
-        aug_neg_transpose_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
-        return cudaGetLastError();
-    }});
-    // b = W - V (cQ) - W (-c P^T)
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, k), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
-    add_gemm(plan, img, pr); pr.clear();
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + k), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
-    add_gemm(plan, img, pr); pr.clear();
-    // C = I + c B U
-    plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * N * B, [=](cudaStream_t s) {
-        aug_add_identity_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(Aug, N, ld, aug_stride);
-        return cudaGetLastError();
-    }});
-    // y = [W^T b; -V^T b] into the right-hand columns (split-K sums)
-    for (int i = 0; i < B; ++i) {
-        pr.push_back(gemm(Wm(i, true), bm(i), Ai(i) + N, ld, true, nullptr, 0, false, k, k, n, 1.f, 0.f));
-        pr.push_back(gemm(Vm(i, true), bm(i), Ai(i) + k * ld + N, ld, true, nullptr, 0, false, k, k, n, -1.f, 0.f));
-    }
-    add_gemm_splitk(plan, img, pr, part); pr.clear();
     // Gaussian elimination with partial pivoting on [C | y], fp64, two levels: 128-column
     // block columns factorised with nb-wide panels (updates confined to the block column),
     // then one row-swap + unit-lower solve over the trailing columns and one K = 128
@@ -601,6 +593,267 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
             add_gemm(plan, img, pr, true); pr.clear();
         }
     }
+}
+
+// ---------------------------------------------------------------- tensor-core plan
+// fp32 products on the tensor cores: each fp32 operand is held as three bf16 planes and a
+// product is the sum of the six plane products with indices summing to <= 2 (the dropped
+// ones are below 2^-24 of the result), accumulated in fp32 TMEM.
+struct Planes {
+    __nv_bfloat16* p;   // 3 contiguous planes of rows x cols
+    int rows, cols;
+};
+struct TcOperand {
+    const CUtensorMap* tm[kTcMaxPlanes];
+    bool mn;
+};
+
+// K-major operand: rows are the M (or N) index, columns the K index; MN-major: rows are K.
+TcOperand tc_operand(TmapPool& pool, const Planes& pl, bool mn) {
+    TcOperand o;
+    o.mn = mn;
+    const size_t plane = static_cast<size_t>(pl.rows) * pl.cols;
+    for (int i = 0; i < kTcMaxPlanes; ++i) o.tm[i] = pool.get(pl.p + i * plane, pl.rows, pl.cols, mn ? 64 : kTcBM / 2);
+    return o;
+}
+
+TcProblem tc_problem(const TcOperand& a, const TcOperand& b, float* out, const float* E, int ld, int M, int N, int K,
+                     float alpha, float beta, bool sym) {
+    TcProblem P;
+    std::memset(&P, 0, sizeof(P));
+    for (int i = 0; i < kTcMaxPlanes; ++i) {
+        P.tmA[i] = a.tm[i];
+        P.tmB[i] = b.tm[i];
+    }
+    P.out[0] = out;
+    P.E[0] = E;
+    P.ld = ld;
+    P.M = M; P.N = N; P.K = K;
+    P.alpha = alpha; P.beta = beta;
+    P.flags = (a.mn ? kProbAMn : 0u) | (b.mn ? kProbBMn : 0u) | (sym ? kProbSym : 0u) | kProbOutF32 |
+              (E != nullptr ? kProbEF32 : 0u);
+    tc_set_segments(P, kTcMaxPlanes, kTcMaxPlanes, 2);
+    return P;
+}
+
+void add_tc(Plan& plan, TableImage& img, const std::vector<TcProblem>& all, unsigned* d_status) {
+    const int sms = device_sm_count();
+    for (size_t first = 0; first < all.size(); first += kMaxTileProblems) {
+        const size_t last = std::min(all.size(), first + static_cast<size_t>(kMaxTileProblems));
+        const std::vector<TcProblem> probs(all.begin() + first, all.begin() + last);
+        std::vector<uint32_t> tiles;
+        double flops = 0;
+        for (size_t p = 0; p < probs.size(); ++p) {
+            const TcProblem& P = probs[p];
+            const int mbs = (P.M + kTcBM - 1) / kTcBM, nbs = (P.N + kTcBN - 1) / kTcBN;
+            const bool sym = (P.flags & kProbSym) != 0;
+            for (int nb = 0; nb < nbs; ++nb)
+                for (int mb = 0; mb < mbs; ++mb)
+                    if (!sym || nb >= mb) tiles.push_back(tile_code(static_cast<int>(p), mb, nb));
+            flops += (sym ? 1.0 : 2.0) * P.M * P.N * P.K;
+        }
+        const TcProblem* dp = img.dev<TcProblem>(img.add(probs.data(), probs.size() * sizeof(TcProblem), kAlign));
+        const uint32_t* dt = img.dev<uint32_t>(img.add(tiles.data(), tiles.size() * sizeof(uint32_t), kAlign));
+        const int nt = static_cast<int>(tiles.size());
+        plan.steps.push_back({MUON_KERNEL_TC_F32, flops, [=](cudaStream_t s) {
+                                  return tc_gemm_launch(dp, dt, nt, d_status, sms, s);
+                              }});
+    }
+}
+
+// Destination of a split-K product: out = alpha * sum of the chunk partials.
+struct SplitTarget {
+    void* out;
+    long long ld;
+    int out_f64;
+    float alpha;
+};
+
+void add_tc_splitk(Plan& plan, TableImage& img, const std::vector<TcProblem>& probs,
+                   const std::vector<SplitTarget>& targets, float* part, unsigned* d_status) {
+    std::vector<TcProblem> chunks;
+    std::vector<SplitKItem> items;
+    long long block0 = 0;
+    float* cur = part;
+    for (size_t p = 0; p < probs.size(); ++p) {
+        const TcProblem& P = probs[p];
+        const int ns = (P.K + kSplitK - 1) / kSplitK;
+        const long long mn = static_cast<long long>(P.M) * P.N;
+        for (int j = 0; j < ns; ++j) {
+            TcProblem C = P;
+            C.k_begin = j * kSplitK;
+            C.K = std::min(kSplitK, P.K - j * kSplitK);
+            C.out[0] = cur + j * mn;
+            C.E[0] = nullptr;
+            C.ld = P.N;
+            C.alpha = 1.f;
+            C.beta = 0.f;
+            C.flags = (P.flags & ~kProbEF32) | kProbOutF32;
+            chunks.push_back(C);
+        }
+        SplitKItem it;
+        std::memset(&it, 0, sizeof(it));
+        it.part = cur; it.out = targets[p].out; it.ld_out = targets[p].ld;
+        it.M = P.M; it.N = P.N; it.nsplit = ns; it.alpha = targets[p].alpha;
+        it.out_f64 = targets[p].out_f64;
+        it.block0 = block0;
+        block0 += (mn + 255) / 256;
+        items.push_back(it);
+        cur += ns * mn;
+    }
+    add_tc(plan, img, chunks, d_status);
+    const SplitKItem* di = img.dev<SplitKItem>(img.add(items.data(), items.size() * sizeof(SplitKItem), kAlign));
+    const int ni = static_cast<int>(items.size());
+    const long long nb = block0;
+    double bytes = 0;
+    for (const auto& it : items) bytes += 4.0 * it.nsplit * it.M * it.N + (it.out_f64 ? 8.0 : 4.0) * it.M * it.N;
+    plan.steps.push_back({MUON_KERNEL_MISC, bytes, [=](cudaStream_t s) {
+                              splitk_reduce_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(di, ni);
+                              return cudaGetLastError();
+                          }});
+}
+
+void add_split3(Plan& plan, TableImage& img, const std::vector<Split3Item>& in) {
+    std::vector<Split3Item> items(in);
+    long long block0 = 0;
+    double bytes = 0;
+    for (auto& it : items) {
+        it.block0 = block0;
+        const long long n = static_cast<long long>(it.rows) * it.cols;
+        block0 += (n + 255) / 256;
+        bytes += n * ((it.src_f64 ? 8.0 : 4.0) + 6.0);
+    }
+    const Split3Item* di = img.dev<Split3Item>(img.add(items.data(), items.size() * sizeof(Split3Item), kAlign));
+    const int ni = static_cast<int>(items.size());
+    const long long nb = block0;
+    plan.steps.push_back({MUON_KERNEL_MISC, bytes, [=](cudaStream_t s) {
+                              split3_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(di, ni);
+                              return cudaGetLastError();
+                          }});
+}
+
+// Appends the projection + Woodbury-Cayley launches for W (batch x n x k) with direction
+// source G (may be the workspace V buffer itself: V = G - W sym(W^T G) is then formed in
+// place, each element read and written by one thread).
+muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, uint8_t* ws, unsigned* d_status,
+                          float* W, const float* G, int batch, int n, int k, float lr, size_t ws_bytes) {
+    // With 16-byte bf16 row pitches, the two products that only shape the direction V (S = W^T G
+    // and V = G - W sym(S)) run on the tensor cores from three bf16 planes.  Every product that
+    // enters C, y, b or the final update stays on the FMA pipes in fp32 with round-to-nearest:
+    // the retraction preserves W^T W = I only as well as those are computed, and the tensor
+    // cores' fp32 accumulation over thousands of MMA steps drifted the 100-step orthogonality
+    // defect to 7e-5 when they carried all products.  A = V W^T - W V^T stays skew for any V,
+    // so the direction's own rounding does not leave the manifold.
+    float* V = reinterpret_cast<float*>(ws + kHeaderBytes + L.V);
+    float* bb = reinterpret_cast<float*>(ws + kHeaderBytes + L.b);
+    float* S = reinterpret_cast<float*>(ws + kHeaderBytes + L.S);
+    double* Aug = reinterpret_cast<double*>(ws + kHeaderBytes + L.Aug);
+    int* piv = reinterpret_cast<int*>(ws + kHeaderBytes + L.piv);
+    float* part = reinterpret_cast<float*>(ws + kHeaderBytes + L.part);
+    const long long nk = static_cast<long long>(n) * k, kk = static_cast<long long>(k) * k;
+    const int N = 2 * k, ncols = 3 * k;
+    const long long ld = ncols, aug_stride = static_cast<long long>(N) * ncols;
+    const float c = 0.5f * lr;
+    const int B = batch;
+    auto Wm = [&](int i, bool t = false) { return Mat{W + i * nk, k, t, false}; };
+    auto Gm = [&](int i) { return Mat{G + i * nk, k, false, false}; };
+    auto Vm = [&](int i, bool t = false) { return Mat{V + i * nk, k, t, false}; };
+    auto bm = [&](int i) { return Mat{bb + i * nk, k, false, false}; };
+    auto Sm = [&](int i) { return Mat{S + i * kk, k, false, false}; };
+    auto Ai = [&](int i) { return Aug + i * aug_stride; };
+    auto Am = [&](int i, long long off) { return Mat{Ai(i) + off, ld, false, true}; };
+
+    std::vector<SimtProblem> pr;
+    const bool tc = L.tc;
+    __nv_bfloat16* planes = tc ? reinterpret_cast<__nv_bfloat16*>(ws + kHeaderBytes + L.planes) : nullptr;
+    TmapPool pool(img);
+    // planes per matrix: W, G (n x k) and S (k x k), three bf16 planes each
+    const size_t per = stiefel_plane_elems(n, k);
+    auto pl = [&](int i, int which) {
+        __nv_bfloat16* base = planes + i * per;
+        if (which < 2) return Planes{base + which * 3 * nk, n, k};
+        return Planes{base + 2 * 3 * nk, k, k};
+    };
+    if (tc) {
+        std::vector<Split3Item> sp;
+        for (int i = 0; i < B; ++i) {
+            for (int which = 0; which < 2; ++which) {
+                Split3Item it;
+                std::memset(&it, 0, sizeof(it));
+                it.src = which == 0 ? static_cast<const void*>(W + i * nk) : static_cast<const void*>(G + i * nk);
+                it.ld = k; it.rows = n; it.cols = k; it.dst = pl(i, which).p;
+                sp.push_back(it);
+            }
+        }
+        add_split3(plan, img, sp);
+        // S = W^T G (split-K over n, fp64 sum of the chunk partials)
+        std::vector<TcProblem> tp;
+        std::vector<SplitTarget> tg;
+        for (int i = 0; i < B; ++i) {
+            tp.push_back(tc_problem(tc_operand(pool, pl(i, 0), true), tc_operand(pool, pl(i, 1), true), nullptr, nullptr,
+                                    k, k, k, n, 1.f, 0.f, false));
+            tg.push_back({S + i * kk, k, 0, 1.f});
+        }
+        add_tc_splitk(plan, img, tp, tg, part, d_status);
+    } else {
+        // S = W^T G (split-K), then sym(S)
+        for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i, true), Gm(i), S + i * kk, k, false, nullptr, 0, false, k, k, n, 1.f, 0.f));
+        add_gemm_splitk(plan, img, pr, part); pr.clear();
+    }
+    plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * kk * B, [=](cudaStream_t s) {
+        symmetrize_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(S, k, kk);
+        return cudaGetLastError();
+    }});
+    // V = G - W sym(S)
+    if (tc) {
+        std::vector<Split3Item> sp;
+        for (int i = 0; i < B; ++i) {
+            Split3Item it;
+            std::memset(&it, 0, sizeof(it));
+            it.src = S + i * kk; it.ld = k; it.rows = k; it.cols = k; it.dst = pl(i, 2).p;
+            sp.push_back(it);
+        }
+        add_split3(plan, img, sp);
+        std::vector<TcProblem> tp;
+        for (int i = 0; i < B; ++i)
+            tp.push_back(tc_problem(tc_operand(pool, pl(i, 0), false), tc_operand(pool, pl(i, 2), true), V + i * nk,
+                                    G + i * nk, k, n, k, k, -1.f, 1.f, false));
+        add_tc(plan, img, tp, d_status);
+    } else {
+        for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Sm(i), V + i * nk, k, false, G + i * nk, k, false, n, k, k, -1.f, 1.f));
+        add_gemm(plan, img, pr); pr.clear();
+    }
+    // fp64 blocks (split-K sums): [0,0] = c P = c W^T V, [0,k] = c Q = c W^T W, [k,0] = -c R = -c V^T V
+    for (int i = 0; i < B; ++i) {
+        pr.push_back(gemm(Wm(i, true), Vm(i), Ai(i), ld, true, nullptr, 0, false, k, k, n, c, 0.f));
+        pr.push_back(gemm(Wm(i, true), Wm(i), Ai(i) + k, ld, true, nullptr, 0, false, k, k, n, c, 0.f));
+        pr.back().sym = 1;                                   // Q = W^T W
+        pr.push_back(gemm(Vm(i, true), Vm(i), Ai(i) + k * ld, ld, true, nullptr, 0, false, k, k, n, -c, 0.f));
+        pr.back().sym = 1;                                   // R = V^T V
+    }
+    add_gemm_splitk(plan, img, pr, part); pr.clear();
+    // [k,k] = -c P^T
+    plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * kk * B, [=](cudaStream_t s) {
+        aug_neg_transpose_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
+        return cudaGetLastError();
+    }});
+    // b = W - V (cQ) - W (-c P^T)
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, k), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + k), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
+    add_gemm(plan, img, pr); pr.clear();
+    // C = I + c B U
+    plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * N * B, [=](cudaStream_t s) {
+        aug_add_identity_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(Aug, N, ld, aug_stride);
+        return cudaGetLastError();
+    }});
+    // y = [W^T b; -V^T b] into the right-hand columns (split-K sums)
+    for (int i = 0; i < B; ++i) {
+        pr.push_back(gemm(Wm(i, true), bm(i), Ai(i) + N, ld, true, nullptr, 0, false, k, k, n, 1.f, 0.f));
+        pr.push_back(gemm(Vm(i, true), bm(i), Ai(i) + k * ld + N, ld, true, nullptr, 0, false, k, k, n, -1.f, 0.f));
+    }
+    add_gemm_splitk(plan, img, pr, part); pr.clear();
+    add_lu_solve(plan, img, Aug, piv, N, ncols, k, B, ld, aug_stride, d_status);
     // W_new = b - c V z_top - c W z_bot, then copy into W
     for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
     add_gemm(plan, img, pr); pr.clear();

@@ -50,18 +50,10 @@ __device__ __forceinline__ TileInfo decode(uint32_t code) {
     return t;
 }
 
-// Segments of the K loop: (A plane, B plane) = (hi,hi), then (hi,lo), (lo,hi) when present.
-__device__ __forceinline__ int num_segments(const TcProblem& P) {
-    return 1 + (P.tmB[1] != nullptr) + (P.tmA[1] != nullptr);
-}
 __device__ __forceinline__ void segment_planes(const TcProblem& P, int seg, int& pa, int& pb) {
-    pa = 0;
-    pb = 0;
-    if (seg == 1) {
-        if (P.tmB[1] != nullptr) pb = 1; else pa = 1;
-    } else if (seg == 2) {
-        pa = 1;
-    }
+    const uint32_t c = (P.segs >> (4 * seg)) & 0xFu;
+    pa = static_cast<int>(c & 3u);
+    pb = static_cast<int>(c >> 2);
 }
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
@@ -71,13 +63,6 @@ __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v)
     w.z = pack_bf16x2(v[4], v[5]);
     w.w = pack_bf16x2(v[6], v[7]);
     *reinterpret_cast<uint4*>(dst) = w;
-}
-__device__ __forceinline__ void load_bf16x8_add(const __nv_bfloat16* src, float* e) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(src));
-    e[0] += bf16_lo_to_f32(w.x); e[1] += bf16_hi_to_f32(w.x);
-    e[2] += bf16_lo_to_f32(w.y); e[3] += bf16_hi_to_f32(w.y);
-    e[4] += bf16_lo_to_f32(w.z); e[5] += bf16_hi_to_f32(w.z);
-    e[6] += bf16_lo_to_f32(w.w); e[7] += bf16_hi_to_f32(w.w);
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTcThreads, 1)
@@ -134,7 +119,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const TileInfo ti = decode(tiles[t]);
             const TcProblem& P = probs[ti.p];
             if (ti.p != last_p) {
-                for (int i = 0; i < 2; ++i) {
+                for (int i = 0; i < kTcMaxPlanes; ++i) {
                     if (P.tmA[i]) tmap_acquire(P.tmA[i]);
                     if (P.tmB[i]) tmap_acquire(P.tmB[i]);
                 }
@@ -145,7 +130,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const int am0 = ti.m0 + HM * static_cast<int>(rank);
             const int bn0 = ti.n0 + HN * static_cast<int>(rank);
             const int kblocks = (P.K + BK - 1) / BK;
-            const int nseg = num_segments(P);
+            const int nseg = P.nseg;
             for (int seg = 0; seg < nseg && ok; ++seg) {
                 int pa, pb;
                 segment_planes(P, seg, pa, pb);
@@ -155,7 +140,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, dev_status)) { ok = false; break; }
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
-                    const int k0 = kb * BK;
+                    const int k0 = P.k_begin + kb * BK;
                     const uint32_t fb = full_leader + stage * 8u;
                     if (rank == 0) {
                         mbar_arrive_expect_tx(&full_bar[stage], PAIR_STAGE_BYTES);
@@ -200,7 +185,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const bool b_mn = (P.flags & kProbBMn) != 0;
             const uint32_t idesc = idesc_bf16_f32(BM, BN, a_mn, b_mn);
             const int kblocks = (P.K + BK - 1) / BK;
-            const int nseg = num_segments(P);
+            const int nseg = P.nseg;
             if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, dev_status)) { ok = false; break; }
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
@@ -237,8 +222,8 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
         // 8 warps: warp & 3 selects the TMEM lane quarter (rows), (warp - 4) >> 2 the half of
-        // the 256 columns.  E (the a*X or b*A operand) is prefetched one 32-column chunk
-        // ahead, the first chunk before waiting for the accumulator.
+        // the 256 columns.  E (the a*X / b*A / fp32 addend) is prefetched one 32-column
+        // chunk ahead as raw 16-byte words, the first chunk before the accumulator wait.
         const int q = warp & 3;
         const int c_beg = ((warp - 4) >> 2) * (BN / 64);
         const int c_end = c_beg + BN / 64;
@@ -254,27 +239,40 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const float alpha = P.alpha * f;
             const float beta = P.beta * f;
             const bool sym = (P.flags & kProbSym) != 0;
+            const bool out_f32 = (P.flags & kProbOutF32) != 0;
+            const bool e_f32 = (P.flags & kProbEF32) != 0;
             const int row = ti.m0 + HM * static_cast<int>(rank) + q * 32 + lane;
             const bool row_ok = row < P.M;
             const bool has_e = (beta != 0.0f) && (P.E[0] != nullptr);
-            const bool e_lo = has_e && (P.E[1] != nullptr);
-            const bool lo_out = P.out[1] != nullptr;
+            const bool e_lo = has_e && !e_f32 && (P.E[1] != nullptr);
+            const bool lo_out = !out_f32 && P.out[1] != nullptr;
             const size_t row_base = static_cast<size_t>(row) * P.ld;
-            // E of chunk c for this row (zero where not needed or out of range)
-            auto load_e = [&](int c, uint4 (&eh)[4], uint4 (&el)[4]) {
+            // E of chunk c for this row: bf16 -> ew[0..3] plane 0, ew[4..7] plane 1; fp32 -> ew[0..7]
+            auto load_e = [&](int c, uint4 (&ew)[8]) {
                 const int col0 = ti.n0 + c * 32;
                 const bool need = has_e && row_ok && col0 < P.N && (!sym || col0 + 31 >= row);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const bool ok = need && (col0 + 8 * g < P.N);
-                    eh[g] = ok ? __ldg(reinterpret_cast<const uint4*>(P.E[0] + row_base + col0 + 8 * g))
-                               : make_uint4(0, 0, 0, 0);
-                    el[g] = (ok && e_lo) ? __ldg(reinterpret_cast<const uint4*>(P.E[1] + row_base + col0 + 8 * g))
-                                         : make_uint4(0, 0, 0, 0);
+                for (int g = 0; g < 8; ++g) ew[g] = make_uint4(0, 0, 0, 0);
+                if (!need) return;
+                if (e_f32) {
+                    const float* e0 = static_cast<const float*>(P.E[0]) + row_base + col0;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        if (col0 + 4 * g < P.N) ew[g] = __ldg(reinterpret_cast<const uint4*>(e0 + 4 * g));
+                } else {
+                    const __nv_bfloat16* e0 = static_cast<const __nv_bfloat16*>(P.E[0]) + row_base + col0;
+                    const __nv_bfloat16* e1 = static_cast<const __nv_bfloat16*>(P.E[1]) + row_base + col0;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        if (col0 + 8 * g < P.N) {
+                            ew[g] = __ldg(reinterpret_cast<const uint4*>(e0 + 8 * g));
+                            if (e_lo) ew[4 + g] = __ldg(reinterpret_cast<const uint4*>(e1 + 8 * g));
+                        }
+                    }
                 }
             };
-            uint4 eh[4], el[4];
-            load_e(c_beg, eh, el);
+            uint4 ew[8];
+            load_e(c_beg, ew);
             if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
@@ -284,42 +282,70 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                 if (col0 >= P.N) break;  // uniform across the warp
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(t_row + c * 32, r);
-                uint4 nh[4], nl[4];
-                if (c + 1 < c_end) load_e(c + 1, nh, nl);
+                uint4 nw[8];
+                if (c + 1 < c_end) load_e(c + 1, nw);
                 tmem_ld_wait();
                 // Rows whose whole chunk lies below the diagonal store nothing.
                 const bool any_store = row_ok && (!sym || col0 + 31 >= row);
                 float v[32];
+                if (e_f32) {
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const uint32_t hw[4] = {eh[g].x, eh[g].y, eh[g].z, eh[g].w};
-                    const uint32_t lw[4] = {el[g].x, el[g].y, el[g].z, el[g].w};
+                    for (int g = 0; g < 8; ++g) {
+                        const uint32_t w4[4] = {ew[g].x, ew[g].y, ew[g].z, ew[g].w};
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float e0 = bf16_lo_to_f32(hw[h]) + bf16_lo_to_f32(lw[h]);
-                        const float e1 = bf16_hi_to_f32(hw[h]) + bf16_hi_to_f32(lw[h]);
-                        v[8 * g + 2 * h] = fmaf(beta, e0, alpha * __uint_as_float(r[8 * g + 2 * h]));
-                        v[8 * g + 2 * h + 1] = fmaf(beta, e1, alpha * __uint_as_float(r[8 * g + 2 * h + 1]));
+                        for (int h = 0; h < 4; ++h)
+                            v[4 * g + h] = fmaf(beta, __uint_as_float(w4[h]), alpha * __uint_as_float(r[4 * g + h]));
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const uint32_t hw[4] = {ew[g].x, ew[g].y, ew[g].z, ew[g].w};
+                        const uint32_t lw[4] = {ew[4 + g].x, ew[4 + g].y, ew[4 + g].z, ew[4 + g].w};
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const float e0 = bf16_lo_to_f32(hw[h]) + bf16_lo_to_f32(lw[h]);
+                            const float e1 = bf16_hi_to_f32(hw[h]) + bf16_hi_to_f32(lw[h]);
+                            v[8 * g + 2 * h] = fmaf(beta, e0, alpha * __uint_as_float(r[8 * g + 2 * h]));
+                            v[8 * g + 2 * h + 1] = fmaf(beta, e1, alpha * __uint_as_float(r[8 * g + 2 * h + 1]));
+                        }
                     }
                 }
                 if (any_store) {
+                    if (out_f32) {
+                        float* o = static_cast<float*>(P.out[0]) + row_base;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int cg = col0 + 8 * g;
-                        if (cg >= P.N) continue;
-                        float lo[8];
+                        for (int g = 0; g < 8; ++g) {
+                            const int cg = col0 + 4 * g;
+                            if (cg >= P.N) continue;
+                            if (!sym || cg >= row) {
+                                *reinterpret_cast<float4*>(o + cg) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                            } else if (cg + 3 >= row) {
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            lo[j] = v[8 * g + j] - __bfloat162float(__float2bfloat16_rn(v[8 * g + j]));
-                        if (!sym || cg >= row) {
-                            store_bf16x8(P.out[0] + row_base + cg, v + 8 * g);
-                            if (lo_out) store_bf16x8(P.out[1] + row_base + cg, lo);
-                        } else if (cg + 7 >= row) {
+                                for (int j = 0; j < 4; ++j)
+                                    if (cg + j >= row) o[cg + j] = v[4 * g + j];
+                            }
+                        }
+                    } else {
+                        __nv_bfloat16* o0 = static_cast<__nv_bfloat16*>(P.out[0]) + row_base;
+                        __nv_bfloat16* o1 = static_cast<__nv_bfloat16*>(P.out[1]) + row_base;
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                if (cg + j >= row) {
-                                    P.out[0][row_base + cg + j] = __float2bfloat16_rn(v[8 * g + j]);
-                                    if (lo_out) P.out[1][row_base + cg + j] = __float2bfloat16_rn(lo[j]);
+                        for (int g = 0; g < 4; ++g) {
+                            const int cg = col0 + 8 * g;
+                            if (cg >= P.N) continue;
+                            float lo[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                lo[j] = v[8 * g + j] - __bfloat162float(__float2bfloat16_rn(v[8 * g + j]));
+                            if (!sym || cg >= row) {
+                                store_bf16x8(o0 + cg, v + 8 * g);
+                                if (lo_out) store_bf16x8(o1 + cg, lo);
+                            } else if (cg + 7 >= row) {
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    if (cg + j >= row) {
+                                        o0[cg + j] = __float2bfloat16_rn(v[8 * g + j]);
+                                        if (lo_out) o1[cg + j] = __float2bfloat16_rn(lo[j]);
+                                    }
                                 }
                             }
                         }
@@ -327,23 +353,25 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                 }
                 if (sym) {
                     // Mirror: element (row, col) with col > row also goes to (col, row).  For a
-                    // fixed col the 32 lanes write 32 consecutive rows: one 64-byte segment.
+                    // fixed col the 32 lanes write 32 consecutive rows: one contiguous segment.
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int col = col0 + j;
                         if (row_ok && col > row && col < P.N) {
                             const size_t off = static_cast<size_t>(col) * P.ld + row;
-                            const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
-                            P.out[0][off] = hv;
-                            if (lo_out) P.out[1][off] = __float2bfloat16_rn(v[j] - __bfloat162float(hv));
+                            if (out_f32) {
+                                static_cast<float*>(P.out[0])[off] = v[j];
+                            } else {
+                                const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
+                                static_cast<__nv_bfloat16*>(P.out[0])[off] = hv;
+                                if (lo_out)
+                                    static_cast<__nv_bfloat16*>(P.out[1])[off] = __float2bfloat16_rn(v[j] - __bfloat162float(hv));
+                            }
                         }
                     }
                 }
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    eh[g] = nh[g];
-                    el[g] = nl[g];
-                }
+                for (int g = 0; g < 8; ++g) ew[g] = nw[g];
             }
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader + acc * 8u);
