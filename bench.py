@@ -170,7 +170,40 @@ def secondary_measurements(only=None):
         out.update(_stiefel(gen))
     if only in (None, "single"):
         out.update(_single())
+    if only == "cublas":
+        out.update(_cublas_reference())
     return out
+
+
+def _cublas_reference():
+    """Context, not the product path: the library GEMM (torch.matmul -> cuBLAS, bf16, fp32
+    accumulate) on the dense equivalents of one Newton-Schulz iteration of one Llama layer
+    (X X^T, A A, B X for 4 x 4096^2, 3 x 4096x11008), looped for a few seconds so the GPU
+    settles at its power-capped clock.  Dense FLOP/s, and the NS chain time those rates
+    imply for the full 224-matrix set."""
+    import torch
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    shapes = [(4096, 4096)] * 4 + [(4096, 11008)] * 3
+    Xs = [torch.empty(s, dtype=torch.bfloat16, device="cuda").normal_(0, 0.01, generator=gen) for s in shapes]
+    As = [torch.empty((4096, 4096), dtype=torch.bfloat16, device="cuda").normal_(0, 0.01, generator=gen) for _ in shapes]
+
+    def one_iteration():
+        for X, A in zip(Xs, As):
+            torch.matmul(X, X.t())
+            torch.matmul(A, A)
+            torch.matmul(A, X)
+
+    dense = sum(2.0 * 4096 * 4096 * s[1] * 2 + 2.0 * 4096 ** 3 for s in shapes)
+    ms = _time_ms(one_iteration, 5, 5)
+    reps = max(1, int(3000.0 / ms))
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    ms = _time_ms(one_iteration, 0, reps)
+    clk = clocks.stop()
+    return {"cublas_dense_tflops": dense / (ms * 1e-3) / 1e12,
+            "cublas_ns_chain_ms_for_set": ms * 5 * 32,
+            "clocks": clk}
 
 
 def _lowrank():
@@ -276,7 +309,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-secondary", action="store_true", help="skip the other parameter sets")
-    ap.add_argument("--case", default=None, choices=["lowrank", "gpt2", "stiefel", "single"],
+    ap.add_argument("--case", default=None, choices=["lowrank", "gpt2", "stiefel", "single", "cublas"],
                     help="time only one of the other parameter sets (for profiling); prints its figures")
     ap.add_argument("--layers", type=int, default=32,
                     help="Llama-7B layers in the set (32 = the full set; 1 = a profiling-sized case)")

@@ -50,6 +50,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps (up to ~10 ms) until the phase
+// completes instead of spinning, which keeps idle roles from burning issue slots and power.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(10000000u)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity.  `abort` (shared) short-circuits the
 // wait once any role of the CTA has given up; on a new timeout the status word gets
 // kDevErrTimeout and `abort` is raised.
@@ -59,7 +73,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     const unsigned long long t0 = global_ns();
     while (true) {
         if (*abort) return false;
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity)) return true;
         if (global_ns() - t0 > kWaitLimitNs) {
             *abort = 1;
             atomicOr(dev_status, kDevErrTimeout);
