@@ -270,7 +270,15 @@ def center_columns(M):
 def muon_cayley_step(W, G, M0, lr: float, beta: float, center: bool = True):
     """One MuonCayley update in the order of §4.3: EMA momentum, centering, tangent
     projection of the centred momentum, Cayley retraction (Woodbury form).
-    Returns (W1, M1)."""
+    Returns (W1, M1).
+
+    A wide W (fewer rows than columns) cannot be column-orthonormal; §4.4 and §6.1 say
+    to transpose such a parameter, update it on the manifold and transpose it back.  The
+    whole step then runs on W^T, G^T, M^T (so the centring takes each row's mean of the
+    caller's M) and the results are transposed back: W stays row-orthonormal."""
+    if np.shape(W)[0] < np.shape(W)[1]:
+        W1t, M1t = muon_cayley_step(np.asarray(W).T, np.asarray(G).T, np.asarray(M0).T, lr, beta, center)
+        return W1t.T, M1t.T
     M1 = ema_momentum(M0, G, beta)
     D = center_columns(M1) if center else M1
     V = project_tangent(W, D)

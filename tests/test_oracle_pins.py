@@ -346,3 +346,25 @@ def test_muon_cayley_step_stays_on_manifold_and_reduces_to_stiefel_step():
     G = r.standard_normal((n, k))
     W1, M1 = orc.muon_cayley_step(W, G, np.zeros((n, k)), lr=0.05, beta=0.0, center=False)
     assert np.allclose(W1, orc.stiefel_cayley_step(W, G, 0.05), atol=1e-14) and np.array_equal(M1, G)
+
+
+def test_muon_cayley_step_on_a_wide_parameter_keeps_rows_orthonormal():
+    """§4.4 / §6.1: a parameter with fewer rows than columns is updated as its transpose.
+    Its rows stay orthonormal, and the centring then removes each row's mean: a gradient
+    that is constant along every row has no direction left and leaves W unchanged."""
+    r = workloads.rng(54)
+    rows, cols = 12, 48
+    W = _orth(r, cols, rows).T
+    W0 = W.copy()
+    M = np.zeros((rows, cols))
+    for _ in range(20):
+        G = r.standard_normal((rows, cols))
+        W, M = orc.muon_cayley_step(W, G, M, lr=3e-3, beta=0.9)
+    assert np.max(np.abs(W @ W.T - np.eye(rows))) < 1e-12
+    assert np.max(np.abs(W - W0)) > 1e-3
+    G_rows = r.standard_normal((rows, 1)) @ np.ones((1, cols))
+    W1, M1 = orc.muon_cayley_step(W, G_rows, np.zeros((rows, cols)), lr=0.5, beta=0.0, center=True)
+    assert np.array_equal(M1, G_rows) and np.allclose(W1, W, atol=1e-15)
+    # the same gradient without centring does move W
+    W2, _ = orc.muon_cayley_step(W, G_rows, np.zeros((rows, cols)), lr=0.5, beta=0.0, center=False)
+    assert np.max(np.abs(W2 - W)) > 1e-3
