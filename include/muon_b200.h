@@ -169,14 +169,21 @@ MUON_API muon_status muon_frobenius_prescale_static(const void* X_in, int in_dty
                                                     float* scale_out, void* stream);
 
 /* MuonCayley update ("Muon 在 Stiefel 流形上的精确闭式更新" page, §3.3 and §4.3) for a
- * contiguous batch of column-orthonormal W (n x k fp32, n >= k):
+ * contiguous batch of column-orthonormal W (n x k fp32, n >= k, row-major):
  *   M <- beta*M + (1 - beta)*G                       (EMA momentum, M fp32, in place)
  *   D = M - (column means of M over the n rows)      (center = 1; D = M when center = 0)
  *   W <- Cayley retraction of W along the tangent projection of D, c = lr/2
  * The centering follows the page's printed code (mean over dim 0, i.e. each column's mean);
- * the projection and retraction are those of stiefel_cayley_step, whose workspace size
- * this entry point shares.  Errors as stiefel_cayley_step, plus INVALID_ARG for a null M,
- * a non-finite beta or center not in {0, 1}. */
+ * the projection and retraction are those of stiefel_cayley_step.
+ * A wide batch (n < k: W row-orthonormal) is updated as its transpose, as the page's §4.4
+ * and §6.1 advise: W, G and M keep the caller's n x k layout, the library transposes W and
+ * the momentum into the workspace, runs the step on the k x n transposes (so the centring
+ * removes each row's mean of the caller's M) and writes W back transposed; M is updated in
+ * place as above.  The workspace then also holds the two transposes.
+ * Errors: INVALID_ARG for null pointers, batch or sizes <= 0, a non-finite lr or beta, or
+ * center not in {0, 1}; UNSUPPORTED_SHAPE when min(n, k) > 4096; ALIGNMENT for W, G or M
+ * not 16-byte aligned or a workspace not 256-byte aligned; WORKSPACE_TOO_SMALL below
+ * muon_cayley_workspace_size (which returns 0 for unsupported arguments). */
 MUON_API size_t muon_cayley_workspace_size(int batch, int n, int k);
 MUON_API muon_status muon_cayley_step(float* W, const float* G, float* M, int batch, int n, int k, float lr,
                                       float beta, int center, void* workspace, size_t ws_bytes, void* stream);

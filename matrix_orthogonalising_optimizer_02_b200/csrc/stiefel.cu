@@ -91,6 +91,26 @@ __global__ void center_kernel(const float* __restrict__ M, const double* __restr
     }
 }
 
+// Batched fp32 transpose, out[b] (cols x rows) = in[b]^T with in[b] rows x cols: 32 x 32
+// tiles staged in shared memory (one padding column against bank conflicts) so that both
+// the reads and the writes are row-contiguous.  Block 32 x 8, grid
+// (ceil(cols/32), ceil(rows/32), batch).
+__global__ void __launch_bounds__(256) transpose_kernel(const float* __restrict__ in, float* __restrict__ out,
+                                                        int rows, int cols) {
+    __shared__ float t[32][33];
+    const long long off = static_cast<long long>(blockIdx.z) * rows * cols;
+    const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int r = r0 + i, c = c0 + threadIdx.x;
+        if (r < rows && c < cols) t[i][threadIdx.x] = in[off + static_cast<long long>(r) * cols + c];
+    }
+    __syncthreads();
+    for (int i = threadIdx.y; i < 32; i += 8) {
+        const int c = c0 + i, r = r0 + threadIdx.x;
+        if (c < cols && r < rows) out[off + static_cast<long long>(c) * rows + r] = t[threadIdx.x][i];
+    }
+}
+
 // out = alpha * sum_j part_j + beta * E, the chunk partials summed in fp64 in order j = 0..
 struct SplitKItem {
     const float* part;   // nsplit consecutive M x N fp32 partials
@@ -231,35 +251,117 @@ lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int 
     }
 }
 
-// For each column c >= j0 + nb: apply the panel's row swaps in order, then solve the unit
-// lower nb x nb triangle L11 (U12 = L11^-1 A12).
-__global__ void lu_swap_trsm_kernel(double* Aug, long long ld, long long stride, int j0, int nb, int ncols,
-                                    const int* piv, long long piv_stride) {
-    extern __shared__ double L[];   // nb x nb
-    double* a = Aug + blockIdx.y * stride;
-    const int* pv = piv + blockIdx.y * piv_stride;
-    for (int e = threadIdx.x; e < nb * nb; e += blockDim.x) {
-        const int i = e / nb, j = e % nb;
-        L[e] = a[(j0 + static_cast<long long>(i)) * ld + j0 + j];
+// Triangular solves on right-hand columns held in registers.  Each column is shared by G
+// consecutive lanes of a warp: lane h of the group holds rows G*m + h (m < R/G), so every
+// lane keeps R/G values and all indices are compile-time.  The triangle sits in shared
+// memory column by column (element (i, l) at T[l * P + i]), zero beyond its live size, so
+// padded rows stay zero.  Both solves are right-looking: once x_l is final its owner lane
+// hands it to the group (one shuffle) and all remaining rows take its term at once.
+template <int R, int G, int P>
+__device__ __forceinline__ void solve_unit_lower(double (&x)[R / G], const double* __restrict__ T, int h) {
+    const int lane = threadIdx.x & 31;
+    const double* Th = T + h;
+#pragma unroll
+    for (int l = 0; l < R - 1; ++l) {
+        const double xl = __shfl_sync(0xffffffffu, x[l / G], (lane & ~(G - 1)) | (l % G));
+#pragma unroll
+        for (int m = 0; m < R / G; ++m) {
+            if (G * m + G - 1 <= l) continue;               // all rows of slot m are at or above l
+            if (G * m > l || h > l - G * m) x[m] = fma(-Th[l * P + G * m], xl, x[m]);
+        }
     }
-    __syncthreads();
-    const int c = j0 + nb + blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= ncols) return;
-    for (int i = 0; i < nb; ++i) {
-        const int p = pv[j0 + i];
-        if (p != j0 + i) {
-            const double t = a[(j0 + static_cast<long long>(i)) * ld + c];
-            a[(j0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
+}
+// Upper triangle; dinv holds the reciprocals of its diagonal (zero on padded rows).
+template <int R, int G, int P>
+__device__ __forceinline__ void solve_upper(double (&x)[R / G], const double* __restrict__ T,
+                                            const double* __restrict__ dinv, int h) {
+    const int lane = threadIdx.x & 31;
+    const double* Th = T + h;
+#pragma unroll
+    for (int l = R - 1; l >= 0; --l) {
+        if (h == l % G) x[l / G] *= dinv[l];
+        const double xl = __shfl_sync(0xffffffffu, x[l / G], (lane & ~(G - 1)) | (l % G));
+#pragma unroll
+        for (int m = 0; m < R / G; ++m) {
+            if (G * m >= l) continue;                       // all rows of slot m are at or below l
+            if (G * m + G - 1 < l || h < l - G * m) x[m] = fma(-Th[l * P + G * m], xl, x[m]);
+        }
+    }
+}
+
+// Copies the w x w block at (r0, r0) of a into T column by column (pitch P, zero-padded to
+// R x R); reads run along rows of a.
+template <int R, int P>
+__device__ __forceinline__ void load_block_cols(double* T, const double* a, long long ld, int r0, int w) {
+    for (int e = threadIdx.x; e < R * R; e += blockDim.x) {
+        const int i = e / R, l = e % R;
+        T[l * P + i] = (i < w && l < w) ? a[(r0 + static_cast<long long>(i)) * ld + r0 + l] : 0.0;
+    }
+}
+
+// Lane h's rows r0 + G*m + h (< r0 + w) of the column starting at p (pitch ld), zero beyond.
+template <int R, int G>
+__device__ __forceinline__ void load_column(double (&x)[R / G], const double* p, long long ld, int w, int h) {
+    p += h * ld;
+#pragma unroll
+    for (int m = 0; m < R / G; ++m) {
+        x[m] = G * m + h < w ? *p : 0.0;
+        p += G * ld;
+    }
+}
+template <int R, int G>
+__device__ __forceinline__ void store_column(const double (&x)[R / G], double* p, long long ld, int w, int h) {
+    p += h * ld;
+#pragma unroll
+    for (int m = 0; m < R / G; ++m) {
+        if (G * m + h < w) *p = x[m];
+        p += G * ld;
+    }
+}
+
+// Applies the row interchanges of rows r0..r0+w-1 (in order) to column c.
+__device__ __forceinline__ void apply_swaps(double* a, long long ld, const int* pv, int r0, int w, int c) {
+    for (int i = 0; i < w; ++i) {
+        const int p = pv[r0 + i];
+        if (p != r0 + i) {
+            const double t = a[(r0 + static_cast<long long>(i)) * ld + c];
+            a[(r0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
             a[static_cast<long long>(p) * ld + c] = t;
         }
     }
-    double x[32];
-    for (int i = 0; i < nb; ++i) {
-        double v = a[(j0 + static_cast<long long>(i)) * ld + c];
-        for (int l = 0; l < i; ++l) v = fma(-L[i * nb + l], x[l], v);
-        x[i] = v;
-        a[(j0 + static_cast<long long>(i)) * ld + c] = v;
-    }
+}
+
+// Row swaps then unit-lower solve U12 = L11^-1 A12 with the w x w triangle at (r0, r0), for
+// the columns [c_lo, ncols) -- (128 / G) columns per block of 128 threads.  The group's
+// first lane applies the swaps; every lane of a warp reaches the shuffles.
+template <int R, int G>
+__device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const int* pv, int r0, int w, int c_lo,
+                                                int ncols, double* T) {
+    constexpr int P = R + 2;
+    load_block_cols<R, P>(T, a, ld, r0, w);
+    __syncthreads();
+    const int c = c_lo + static_cast<int>(blockIdx.x) * (128 / G) + static_cast<int>(threadIdx.x) / G;
+    const int h = static_cast<int>(threadIdx.x) % G;
+    const bool live = c < ncols;
+    if (live && h == 0) apply_swaps(a, ld, pv, r0, w, c);
+    __syncwarp();
+    double* col = a + (live ? c : c_lo) + r0 * ld;
+    const int wl = live ? w : 0;
+    double x[R / G];
+    load_column<R, G>(x, col, ld, wl, h);
+    solve_unit_lower<R, G, P>(x, T, h);
+    store_column<R, G>(x, col, ld, wl, h);
+}
+
+// For each column c in [j0 + nb, ncols): apply the panel's row swaps in order, then solve
+// the unit-lower nb x nb triangle L11 (U12 = L11^-1 A12).  nb <= kPanelMax.
+constexpr int kPanelMax = 32, kPanelLanes = 2;
+__global__ void __launch_bounds__(128)
+lu_swap_trsm_kernel(double* Aug, long long ld, long long stride, int j0, int nb, int ncols, const int* piv,
+                    long long piv_stride) {
+    __shared__ __align__(16) double T[kPanelMax * (kPanelMax + 2)];
+    swap_trsm_block<kPanelMax, kPanelLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, j0, nb,
+                                            j0 + nb, ncols, T);
 }
 
 // Within the current block column: apply the row swaps of panel rows j0..j0+w-1 to the
@@ -282,63 +384,42 @@ __global__ void lu_swap_cols_kernel(double* Aug, long long ld, long long stride,
 
 // After a block column J0..J0+JB-1 is factorised: for every column c >= c_lo, apply the
 // block's JB row swaps in order, then solve with the JB x JB unit-lower L11 (U12 = L11^-1 A12).
-constexpr int kLuBlock = 128;
+constexpr int kLuBlock = 64, kLuLanes = 4;
 __global__ void __launch_bounds__(128)
 lu_block_swap_trsm_kernel(double* Aug, long long ld, long long stride, int J0, int JB, int c_lo, int ncols,
                           const int* piv, long long piv_stride) {
-    extern __shared__ double Lb[];   // JB x JB
-    double* a = Aug + blockIdx.y * stride;
-    const int* pv = piv + blockIdx.y * piv_stride;
-    for (int e = threadIdx.x; e < JB * JB; e += blockDim.x) {
-        const int i = e / JB, j = e % JB;
-        Lb[e] = a[(J0 + static_cast<long long>(i)) * ld + J0 + j];
-    }
-    __syncthreads();
-    const int c = c_lo + blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= ncols) return;
-    for (int i = 0; i < JB; ++i) {
-        const int p = pv[J0 + i];
-        if (p != J0 + i) {
-            const double t = a[(J0 + static_cast<long long>(i)) * ld + c];
-            a[(J0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
-            a[static_cast<long long>(p) * ld + c] = t;
-        }
-    }
-    double x[kLuBlock];
-    for (int i = 0; i < JB; ++i) {
-        double v = a[(J0 + static_cast<long long>(i)) * ld + c];
-        for (int l = 0; l < i; ++l) v = fma(-Lb[i * JB + l], x[l], v);
-        x[i] = v;
-        a[(J0 + static_cast<long long>(i)) * ld + c] = v;
-    }
+    __shared__ __align__(16) double T[kLuBlock * (kLuBlock + 2)];
+    swap_trsm_block<kLuBlock, kLuLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, J0, JB, c_lo,
+                                        ncols, T);
 }
 
 // Back substitution on one diagonal block: rows i0..i0+bs-1 of the right-hand columns
-// (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows).
-constexpr int kBackBlock = 64;
-__global__ void back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, int rhs0, int nrhs) {
-    __shared__ double U[kBackBlock * kBackBlock];
+// (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows); 32 columns per block.
+constexpr int kBackBlock = 64, kBackLanes = 4, kBackPitch = kBackBlock + 2;
+__global__ void __launch_bounds__(128)
+back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, int rhs0, int nrhs) {
+    __shared__ __align__(16) double T[kBackBlock * kBackPitch];
+    __shared__ double dinv[kBackBlock];
     double* a = Aug + blockIdx.y * stride;
-    for (int e = threadIdx.x; e < bs * bs; e += blockDim.x) {
-        const int i = e / bs, j = e % bs;
-        U[i * kBackBlock + j] = a[(i0 + static_cast<long long>(i)) * ld + i0 + j];
-    }
+    load_block_cols<kBackBlock, kBackPitch>(T, a, ld, i0, bs);
+    for (int l = threadIdx.x; l < kBackBlock; l += blockDim.x)
+        dinv[l] = l < bs ? 1.0 / a[(i0 + static_cast<long long>(l)) * ld + i0 + l] : 0.0;
     __syncthreads();
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= nrhs) return;
-    double x[kBackBlock];
-    for (int i = bs - 1; i >= 0; --i) {
-        double v = a[(i0 + static_cast<long long>(i)) * ld + rhs0 + c];
-        for (int l = i + 1; l < bs; ++l) v = fma(-U[i * kBackBlock + l], x[l], v);
-        x[i] = v / U[i * kBackBlock + i];
-        a[(i0 + static_cast<long long>(i)) * ld + rhs0 + c] = x[i];
-    }
+    const int c = static_cast<int>(blockIdx.x) * (128 / kBackLanes) + static_cast<int>(threadIdx.x) / kBackLanes;
+    const int h = static_cast<int>(threadIdx.x) % kBackLanes;
+    const bool live = c < nrhs;
+    double* col = a + rhs0 + (live ? c : 0) + i0 * ld;
+    const int wl = live ? bs : 0;
+    double x[kBackBlock / kBackLanes];
+    load_column<kBackBlock, kBackLanes>(x, col, ld, wl, h);
+    solve_upper<kBackBlock, kBackLanes, kBackPitch>(x, T, dinv, h);
+    store_column<kBackBlock, kBackLanes>(x, col, ld, wl, h);
 }
 
 // Widest panel (<= 32 columns) whose (N x nb) fp64 copy fits in 200 KB of shared memory.
 int lu_panel_width(int N) {
     const int nb = static_cast<int>((200 * 1024) / (static_cast<size_t>(N) * sizeof(double)));
-    return std::max(1, std::min(32, nb));
+    return std::max(1, std::min(kPanelMax, nb));
 }
 
 struct StiefelLayout {
@@ -376,14 +457,34 @@ StiefelLayout stiefel_layout(int batch, int n, int k) {
     return L;
 }
 
+// MuonCayley on a wide parameter (rows < cols) runs on the transpose: the Stiefel layout of
+// the transposed shape plus the transposed W and momentum, ahead of the plan tables.
+struct CayleyLayout {
+    StiefelLayout st;
+    size_t Wt = 0, Mt = 0;
+};
+CayleyLayout cayley_layout(int batch, int rows, int cols) {
+    const bool wide = rows < cols;
+    CayleyLayout C;
+    C.st = stiefel_layout(batch, wide ? cols : rows, wide ? rows : cols);
+    if (wide) {
+        const size_t nk = static_cast<size_t>(rows) * cols * sizeof(float) * batch;
+        C.Wt = C.st.data_bytes;
+        C.Mt = align_up(C.Wt + nk, kAlign);
+        C.st.data_bytes = align_up(C.Mt + nk, kAlign);
+        C.st.table_offset = kHeaderBytes + C.st.data_bytes;
+    }
+    return C;
+}
+
 size_t stiefel_tables_bound(int batch, int n, int k) {
     const int N = 2 * k, nb = lu_panel_width(N);
-    const int panels = (N + nb - 1) / nb;
+    const int outer = (N + kLuBlock - 1) / kLuBlock;
+    const int panels = outer * ((kLuBlock + nb - 1) / nb);   // panels never straddle a block column
     const int back = (N + kBackBlock - 1) / kBackBlock;
     auto tiles = [](long long M, long long Nn) { return ((M + kSimtBM - 1) / kSimtBM) * ((Nn + kSimtBN - 1) / kSimtBN); };
     long long t = 0;
     t += tiles(k, k) * 1 + tiles(n, k) * 1 + tiles(k, k) * 3 + tiles(n, k) * 2 + tiles(k, k) * 2 + tiles(n, k) * 2;
-    const int outer = (N + kLuBlock - 1) / kLuBlock;
     for (int p = 0; p < panels; ++p) t += tiles(N, kLuBlock);
     for (int q = 0; q < outer; ++q) t += tiles(N - q * kLuBlock, 3LL * k - q * kLuBlock);
     for (int q = 0; q < back; ++q) t += tiles(static_cast<long long>(q) * kBackBlock, k);
@@ -538,7 +639,8 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
             if (right_in > 0) {
                 const int block_end = J0 + JB;
                 plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right_in * B, [=](cudaStream_t s) {
-                    lu_swap_trsm_kernel<<<dim3((right_in + 127) / 128, B), 128, static_cast<size_t>(w) * w * sizeof(double), s>>>(
+                    constexpr int cols_per_block = 128 / kPanelLanes;
+                    lu_swap_trsm_kernel<<<dim3((right_in + cols_per_block - 1) / cols_per_block, B), 128, 0, s>>>(
                         Aug, ld, aug_stride, j0, w, block_end, piv, N);
                     return cudaGetLastError();
                 }});
@@ -555,13 +657,8 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
         if (right > 0) {
             const int c_lo = J0 + JB;
             plan.steps.push_back({MUON_KERNEL_LU, 1.0 * JB * JB * right * B, [=](cudaStream_t s) {
-                static bool attr = false;
-                if (!attr) {
-                    cudaFuncSetAttribute(lu_block_swap_trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kLuBlock * kLuBlock * static_cast<int>(sizeof(double)));
-                    attr = true;
-                }
-                lu_block_swap_trsm_kernel<<<dim3((right + 127) / 128, B), 128, static_cast<size_t>(JB) * JB * sizeof(double), s>>>(
+                constexpr int cols_per_block = 128 / kLuLanes;
+                lu_block_swap_trsm_kernel<<<dim3((right + cols_per_block - 1) / cols_per_block, B), 128, 0, s>>>(
                     Aug, ld, aug_stride, J0, JB, c_lo, ncols, piv, N);
                 return cudaGetLastError();
             }});
@@ -581,7 +678,9 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
     for (int q = nblk - 1; q >= 0; --q) {
         const int i0 = q * kBackBlock, bs = std::min(kBackBlock, N - i0);
         plan.steps.push_back({MUON_KERNEL_LU, 1.0 * bs * bs * k * B, [=](cudaStream_t s) {
-            back_diag_kernel<<<dim3((k + 127) / 128, B), 128, 0, s>>>(Aug, ld, aug_stride, i0, bs, N, k);
+            constexpr int cols_per_block = 128 / kBackLanes;
+            back_diag_kernel<<<dim3((k + cols_per_block - 1) / cols_per_block, B), 128, 0, s>>>(Aug, ld, aug_stride, i0,
+                                                                                               bs, N, k);
             return cudaGetLastError();
         }});
         if (i0 > 0) {
@@ -903,7 +1002,13 @@ muon_status stiefel_cayley_step(float* W, const float* G, int batch, int n, int 
     return run_plan(kw.k, workspace, L.table_offset, build, stream);
 }
 
-size_t muon_cayley_workspace_size(int batch, int n, int k) { return stiefel_workspace_size(batch, n, k); }
+size_t muon_cayley_workspace_size(int batch, int n, int k) {
+    if (batch <= 0 || n <= 0 || k <= 0) return 0;
+    const int nt = n < k ? k : n, kt = n < k ? n : k;
+    if (kt > 4096 || nt > kMaxTileBlocks * kSimtBM) return 0;
+    const CayleyLayout C = cayley_layout(batch, n, k);
+    return C.st.table_offset + stiefel_tables_bound(batch, nt, kt);
+}
 
 muon_status muon_cayley_step(float* W, const float* G, float* M, int batch, int n, int k, float lr, float beta,
                              int center, void* workspace, size_t ws_bytes, void* stream_) {
@@ -911,11 +1016,15 @@ muon_status muon_cayley_step(float* W, const float* G, float* M, int batch, int 
     if (W == nullptr || G == nullptr || workspace == nullptr) return MUON_ERR_INVALID_ARG;
     if (batch <= 0 || batch > kMaxTileProblems / 4 || n <= 0 || k <= 0 || !std::isfinite(lr))
         return MUON_ERR_INVALID_ARG;
-    if (n < k || k > 4096 || n > kMaxTileBlocks * kSimtBM) return MUON_ERR_UNSUPPORTED_SHAPE;
+    // A wide parameter (n < k) is updated as its transpose (k x n, column-orthonormal).
+    const bool wide = n < k;
+    const int nt = wide ? k : n, kt = wide ? n : k;
+    if (kt > 4096 || nt > kMaxTileBlocks * kSimtBM) return MUON_ERR_UNSUPPORTED_SHAPE;
     if (!al16(W) || !al16(G) || !al16(M) || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return MUON_ERR_ALIGNMENT;
     if (ws_bytes < muon_cayley_workspace_size(batch, n, k)) return MUON_ERR_WORKSPACE_TOO_SMALL;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    const StiefelLayout L = stiefel_layout(batch, n, k);
+    const CayleyLayout C = cayley_layout(batch, n, k);
+    const StiefelLayout& L = C.st;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     unsigned* d_status = static_cast<unsigned*>(workspace);
 
@@ -927,24 +1036,39 @@ muon_status muon_cayley_step(float* W, const float* G, float* M, int batch, int 
     auto build = [&](Plan& plan, TableImage& img) -> muon_status {
         float* V = reinterpret_cast<float*>(ws + kHeaderBytes + L.V);
         double* cm = center ? reinterpret_cast<double*>(ws + kHeaderBytes + L.cm) : nullptr;
+        float* Wt = wide ? reinterpret_cast<float*>(ws + kHeaderBytes + C.Wt) : W;
+        float* Mt = wide ? reinterpret_cast<float*>(ws + kHeaderBytes + C.Mt) : M;
         const long long total = static_cast<long long>(batch) * n * k;
         const int grid = static_cast<int>(std::min<long long>((total + 255) / 256, 148LL * 16));
         const float b = beta;
+        // transposes of one batch: rows x cols -> cols x rows
+        auto transpose = [&](const float* in, float* out, int rows, int cols) {
+            const dim3 tg((cols + 31) / 32, (rows + 31) / 32, batch);
+            plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * total, [=](cudaStream_t s) {
+                transpose_kernel<<<tg, dim3(32, 8), 0, s>>>(in, out, rows, cols);
+                return cudaGetLastError();
+            }});
+        };
         plan.steps.push_back({MUON_KERNEL_MOMENTUM, 12.0 * total, [=](cudaStream_t s) {
             ema_kernel<<<grid, 256, 0, s>>>(M, G, total, b);
             return cudaGetLastError();
         }});
+        if (wide) transpose(M, Mt, n, k);
         if (cm != nullptr) {
             plan.steps.push_back({MUON_KERNEL_MISC, 4.0 * total, [=](cudaStream_t s) {
-                column_mean_kernel<<<dim3((k + 127) / 128, batch), 128, 0, s>>>(M, cm, n, k);
+                column_mean_kernel<<<dim3((kt + 127) / 128, batch), 128, 0, s>>>(Mt, cm, nt, kt);
                 return cudaGetLastError();
             }});
         }
         plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * total, [=](cudaStream_t s) {
-            center_kernel<<<grid, 256, 0, s>>>(M, cm, V, n, k, total);
+            center_kernel<<<grid, 256, 0, s>>>(Mt, cm, V, nt, kt, total);
             return cudaGetLastError();
         }});
-        return build_stiefel(plan, img, L, ws, d_status, W, V, batch, n, k, lr, ws_bytes);
+        if (wide) transpose(W, Wt, n, k);
+        const muon_status st = build_stiefel(plan, img, L, ws, d_status, Wt, V, batch, nt, kt, lr, ws_bytes);
+        if (st != MUON_OK) return st;
+        if (wide) transpose(Wt, W, k, n);
+        return MUON_OK;
     };
     return run_plan(kw.k, workspace, L.table_offset, build, stream);
 }

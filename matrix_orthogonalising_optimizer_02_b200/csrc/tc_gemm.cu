@@ -37,6 +37,7 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+static_assert(SMEM_TOTAL <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 static_assert(HM == 128 && HN == 128, "pair tile is 256 x 256");
 
 struct TileInfo {

@@ -82,16 +82,17 @@ class Muon(torch.optim.Optimizer):
 
 class MuonCayley(torch.optim.Optimizer):
     """Stiefel-manifold Muon: EMA momentum, column centering, tangent projection and the
-    Cayley retraction in Woodbury form; parameters must be fp32, column-orthonormal,
-    shaped n x k with n >= k."""
+    Cayley retraction in Woodbury form.  Parameters are fp32 and orthonormal along their
+    shorter side: a tall n x k parameter has orthonormal columns, a wide one orthonormal
+    rows and is updated as its transpose inside the library (page §4.4)."""
 
     def __init__(self, params, lr=3e-3, momentum=0.9, center=True):
         super().__init__(params, dict(lr=lr, momentum=momentum, center=center))
         for g in self.param_groups:
             for p in g["params"]:
                 _check_matrix(p)
-                if p.dtype != torch.float32 or p.shape[0] < p.shape[1]:
-                    raise ValueError("MuonCayley needs fp32 n x k parameters with n >= k (transpose otherwise)")
+                if p.dtype != torch.float32:
+                    raise ValueError("MuonCayley needs fp32 parameters")
         self._ws = _Workspaces()
 
     @torch.no_grad()

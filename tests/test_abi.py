@@ -51,6 +51,10 @@ def test_workspace_queries_are_host_only():
     assert mb.ns_workspace_size(1, 1000, 1001, mb.Schedule.fixed(5, fp32_mode=True)) > 0
     assert mb.stiefel_workspace_size(16, 4096, 1024) > 16 * 4096 * 1024 * 8
     assert mb.stiefel_workspace_size(1, 10, 20) == 0            # n < k
+    # MuonCayley takes wide batches: the transposed plan plus the transposes of W and M
+    assert mb.muon_cayley_workspace_size(2, 64, 256) >= mb.stiefel_workspace_size(2, 256, 64) + 2 * 2 * 64 * 256 * 4
+    assert mb.muon_cayley_workspace_size(2, 256, 64) == mb.stiefel_workspace_size(2, 256, 64)
+    assert mb.muon_cayley_workspace_size(1, 5000, 4100) == 0     # min(n, k) > 4096
 
 
 def _descs(shapes, ptr=1 << 20):

@@ -102,3 +102,27 @@ def test_muon_cayley_steps_match_oracle(center):
         assert np.max(np.abs(host(W[i]) - Wr[i])) <= 2e-5
         assert np.max(np.abs(host(M[i]) - Mr[i])) <= 1e-5 * max(1.0, np.max(np.abs(Mr[i])))
         assert orc.orthogonality_error(host(W[i])) <= 1e-5
+
+
+def test_muon_cayley_wide_batch_matches_transposed_oracle():
+    """A wide batch (64 x 256: orthonormal rows) goes through the library's transpose
+    branch; 3 steps against the oracle, which updates the transpose (page §4.4)."""
+    batch, rows, cols, lr, beta = 2, 64, 256, 3e-3, 0.9
+    Ws = np.ascontiguousarray(np.swapaxes(workloads.stiefel_problem(seed=970, batch=batch, n=cols, k=rows), 1, 2))
+    W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+    M = torch.zeros_like(W)
+    ws = mb.workspace(mb.muon_cayley_workspace_size(batch, rows, cols))
+    Wr = [Ws[i].copy() for i in range(batch)]
+    Mr = [np.zeros((rows, cols)) for _ in range(batch)]
+    for step in range(3):
+        Gs = workloads.stiefel_gradient(970, step, batch, rows, cols)
+        G = torch.tensor(Gs, dtype=torch.float32, device="cuda")
+        mb.muon_cayley_step(W, G, M, lr, beta, ws, center=True)
+        for i in range(batch):
+            Wr[i], Mr[i] = orc.muon_cayley_step(Wr[i], Gs[i].astype(np.float64), Mr[i], lr, float(np.float32(beta)))
+    assert mb.device_status(ws) == mb.MUON_OK
+    for i in range(batch):
+        got = host(W[i])
+        assert np.max(np.abs(got - Wr[i])) <= 2e-5
+        assert np.max(np.abs(host(M[i]) - Mr[i])) <= 1e-5 * max(1.0, np.max(np.abs(Mr[i])))
+        assert np.max(np.abs(got @ got.T - np.eye(rows))) <= 1e-5

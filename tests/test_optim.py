@@ -15,8 +15,7 @@ def test_muon_rejects_non_matrices():
         Muon([torch.nn.Parameter(torch.zeros(8))])
     with pytest.raises(ValueError):
         Muon([torch.nn.Parameter(torch.zeros(8, 8))], scale_mode="bogus")
-    with pytest.raises(ValueError):
-        MuonCayley([torch.nn.Parameter(torch.zeros(4, 8))])          # n < k
+    MuonCayley([torch.nn.Parameter(torch.zeros(4, 8))])              # wide: updated as its transpose
     with pytest.raises(ValueError):
         MuonCayley([torch.nn.Parameter(torch.zeros(8, 4, dtype=torch.bfloat16))])
 
