@@ -159,6 +159,52 @@ simt_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
             f = (P.scale_pow == 1) ? s : s * s;
         }
         const float alpha = P.alpha * f, beta = P.beta * f;
+        if constexpr (sizeof(Acc) == sizeof(double)) {
+            // The fp64 kernel's short-K launches (the LU updates) are dominated by this
+            // epilogue.  With an fp64 output and addend on 16-byte aligned rows, each of the
+            // thread's two groups of 4 consecutive columns per row goes as 32-byte accesses,
+            // so a warp touches whole sectors.
+            const bool has_e = beta != 0.f;
+            const bool vec_ok = !P.sym && P.out_f64 && (reinterpret_cast<uintptr_t>(P.out) & 15u) == 0 &&
+                                P.ld_out % 2 == 0 &&
+                                (!has_e || (P.e_f64 && (reinterpret_cast<uintptr_t>(P.E) & 15u) == 0 && P.ld_e % 2 == 0));
+            if (vec_ok) {
+                const double* E = static_cast<const double*>(P.E);
+                double* O = static_cast<double*>(P.out);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+                    if (m >= P.M) continue;
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        const int nq = n0 + g * 64 + tx * 4;
+                        const long long eo = static_cast<long long>(m) * P.ld_e + nq;
+                        const long long oo = static_cast<long long>(m) * P.ld_out + nq;
+                        double v[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) v[j] = static_cast<double>(alpha) * acc[i][4 * g + j];
+                        if (nq + 3 < P.N) {
+                            if (has_e) {
+                                const double2 e0 = *reinterpret_cast<const double2*>(E + eo);
+                                const double2 e1 = *reinterpret_cast<const double2*>(E + eo + 2);
+                                const double b = beta;
+                                v[0] = fma(b, e0.x, v[0]); v[1] = fma(b, e0.y, v[1]);
+                                v[2] = fma(b, e1.x, v[2]); v[3] = fma(b, e1.y, v[3]);
+                            }
+                            *reinterpret_cast<double2*>(O + oo) = make_double2(v[0], v[1]);
+                            *reinterpret_cast<double2*>(O + oo + 2) = make_double2(v[2], v[3]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                if (nq + j >= P.N) continue;
+                                O[oo + j] = has_e ? fma(static_cast<double>(beta), E[eo + j], v[j]) : v[j];
+                            }
+                        }
+                    }
+                }
+                continue;
+            }
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));

@@ -181,29 +181,34 @@ __global__ void split3_kernel(const Split3Item* __restrict__ items, int count) {
 }
 
 // Panel factorisation (partial pivoting) of rows j0..N-1, columns j0..j0+nb-1, held in
-// shared memory.  Records the pivot row of each column in piv (absolute row indices).
+// shared memory column by column with an odd pitch (consecutive rows in consecutive words,
+// so the per-row sweeps are free of bank conflicts).  Records the pivot row of each column
+// in piv (absolute row indices).
+__host__ __device__ constexpr int panel_pitch(int rows) { return rows | 1; }
 __global__ void __launch_bounds__(1024)
 lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int nb, int* piv, long long piv_stride,
                 unsigned* status) {
-    extern __shared__ double pan[];  // (N - j0) x nb
+    extern __shared__ double pan[];  // nb columns of panel_pitch(N - j0)
     __shared__ double red_v[32];
     __shared__ int red_i[32];
     __shared__ int s_p;
     double* a = Aug + blockIdx.x * stride;
     int* pv = piv + blockIdx.x * piv_stride;
     const int rows = N - j0;
+    const int pitch = panel_pitch(rows);
     const int tid = threadIdx.x, nt = blockDim.x;
     for (int e = tid; e < rows * nb; e += nt) {
         const int r = e / nb, c = e % nb;
-        pan[e] = a[(j0 + static_cast<long long>(r)) * ld + j0 + c];
+        pan[c * pitch + r] = a[(j0 + static_cast<long long>(r)) * ld + j0 + c];
     }
     __syncthreads();
     for (int jj = 0; jj < nb; ++jj) {
-        // argmax |pan[r][jj]| over r >= jj (ties: smallest row)
+        const double* colj = pan + jj * pitch;
+        // argmax |pan(r, jj)| over r >= jj (ties: smallest row)
         double best = -1.0;
         int bi = jj;
         for (int r = jj + tid; r < rows; r += nt) {
-            const double v = fabs(pan[r * nb + jj]);
+            const double v = fabs(colj[r]);
             if (v > best) { best = v; bi = r; }
         }
 #pragma unroll
@@ -232,22 +237,23 @@ lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int 
         __syncthreads();
         const int p = s_p;
         if (p != jj && tid < nb) {
-            const double t = pan[jj * nb + tid];
-            pan[jj * nb + tid] = pan[p * nb + tid];
-            pan[p * nb + tid] = t;
+            double* cc = pan + tid * pitch;
+            const double t = cc[jj];
+            cc[jj] = cc[p];
+            cc[p] = t;
         }
         __syncthreads();
-        const double piv_v = pan[jj * nb + jj];
+        const double piv_v = colj[jj];
         for (int r = jj + 1 + tid; r < rows; r += nt) {
-            const double l = pan[r * nb + jj] / piv_v;
-            pan[r * nb + jj] = l;
-            for (int c = jj + 1; c < nb; ++c) pan[r * nb + c] = fma(-l, pan[jj * nb + c], pan[r * nb + c]);
+            const double l = colj[r] / piv_v;
+            pan[jj * pitch + r] = l;
+            for (int c = jj + 1; c < nb; ++c) pan[c * pitch + r] = fma(-l, pan[c * pitch + jj], pan[c * pitch + r]);
         }
         __syncthreads();
     }
     for (int e = tid; e < rows * nb; e += nt) {
         const int r = e / nb, c = e % nb;
-        a[(j0 + static_cast<long long>(r)) * ld + j0 + c] = pan[e];
+        a[(j0 + static_cast<long long>(r)) * ld + j0 + c] = pan[c * pitch + r];
     }
 }
 
@@ -416,9 +422,10 @@ back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, in
     store_column<kBackBlock, kBackLanes>(x, col, ld, wl, h);
 }
 
-// Widest panel (<= 32 columns) whose (N x nb) fp64 copy fits in 200 KB of shared memory.
+// Widest panel (<= 32 columns) whose fp64 copy (nb columns of panel_pitch(N)) fits in 200 KB
+// of shared memory.
 int lu_panel_width(int N) {
-    const int nb = static_cast<int>((200 * 1024) / (static_cast<size_t>(N) * sizeof(double)));
+    const int nb = static_cast<int>((200 * 1024) / (static_cast<size_t>(panel_pitch(N)) * sizeof(double)));
     return std::max(1, std::min(kPanelMax, nb));
 }
 
@@ -616,7 +623,7 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
         const int JB = std::min(kLuBlock, N - J0);
         for (int j0 = J0; j0 < J0 + JB; j0 += nb) {
             const int w = std::min(nb, J0 + JB - j0);
-            const size_t smem = static_cast<size_t>(N - j0) * w * sizeof(double);
+            const size_t smem = static_cast<size_t>(panel_pitch(N - j0)) * w * sizeof(double);
             const double lu_flops = 2.0 * (N - j0) * w * w * B;
             plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
                 static bool attr = false;
