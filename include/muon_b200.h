@@ -127,6 +127,23 @@ MUON_API size_t muon_step_workspace_min(const muon_matrix_desc* descs, int count
 MUON_API muon_status muon_step_batched(const muon_matrix_desc* descs, int count, const muon_hyper* hp,
                               void* workspace, size_t ws_bytes, void* stream);
 
+/* The same step with every G in pinned (page-locked) host memory; W, M and O_out stay on
+ * the device.  The set is cut, in descriptor order, into up to MUON_HOST_GRAD_CHUNKS
+ * chunks of about equal gradient bytes.  The chunks' gradients are copied into two staging
+ * slots of the workspace on a library-owned copy stream, one cudaMemcpyAsync per matrix,
+ * while the previous chunk's step runs on `stream`, so the host-to-device transfer
+ * overlaps the computation of earlier chunks.  Results equal those of muon_step_batched on
+ * device copies of the gradients.  `stream` orders the whole call (the copy stream joins it
+ * through events), so it can be captured in a CUDA graph.  The workspace's device status
+ * word gathers the status of every chunk.  There is no counterpart of this entry point on
+ * the source pages: it serves callers whose gradients arrive in host memory.
+ * Errors: those of muon_step_batched; INVALID_ARG if a G is not page-locked host memory.
+ * Query the workspace size with muon_step_host_grad_workspace_size (0 if invalid). */
+#define MUON_HOST_GRAD_CHUNKS 8
+MUON_API size_t muon_step_host_grad_workspace_size(const muon_matrix_desc* descs, int count, const muon_hyper* hp);
+MUON_API muon_status muon_step_batched_host_grad(const muon_matrix_desc* descs, int count, const muon_hyper* hp,
+                                                 void* workspace, size_t ws_bytes, void* stream);
+
 /* Newton-Schulz orthogonalisation (Muon optimizer page, zeropower_via_newtonschulz) of a
  * contiguous batch of rows x cols matrices: X_out[i] ~ msign(X_in[i]).  X_in is read as
  * in_dtype; in bf16 mode an fp32 input is first rounded to bf16 (the page's cast).

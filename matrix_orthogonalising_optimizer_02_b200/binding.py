@@ -31,7 +31,8 @@ EXPORTED = (
     "ns_workspace_size", "ns_orthogonalize", "stiefel_workspace_size", "stiefel_cayley_step",
     "muon_workspace_device_status", "muon_timing_enable", "muon_timing_reset", "muon_timing_read",
     "muon_status_string", "muon_build_info", "muon_frobenius_prescale_static",
-    "muon_cayley_workspace_size", "muon_cayley_step",
+    "muon_cayley_workspace_size", "muon_cayley_step", "muon_step_host_grad_workspace_size",
+    "muon_step_batched_host_grad",
 )
 
 
@@ -71,6 +72,9 @@ def _lib():
         "muon_step_workspace_size": (c_size_t, [POINTER(MatrixDesc), c_int, POINTER(Hyper)]),
         "muon_step_workspace_min": (c_size_t, [POINTER(MatrixDesc), c_int, POINTER(Hyper)]),
         "muon_step_batched": (c_int, [POINTER(MatrixDesc), c_int, POINTER(Hyper), c_void_p, c_size_t, c_void_p]),
+        "muon_step_host_grad_workspace_size": (c_size_t, [POINTER(MatrixDesc), c_int, POINTER(Hyper)]),
+        "muon_step_batched_host_grad": (c_int, [POINTER(MatrixDesc), c_int, POINTER(Hyper), c_void_p, c_size_t,
+                                                c_void_p]),
         "ns_workspace_size": (c_size_t, [c_int, c_int, c_int, POINTER(NsSchedule)]),
         "ns_orthogonalize": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, POINTER(NsSchedule),
                                      c_void_p, c_size_t, c_void_p]),
@@ -187,6 +191,21 @@ def muon_step_batched(mats: Sequence[Matrix], hp, workspace, stream=None):
     st = _lib().muon_step_batched(_descs(mats), len(mats), ctypes.byref(hp[0]), workspace.data_ptr(),
                                   workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "muon_step_batched")
+
+
+def muon_step_host_grad_workspace_size(mats: Sequence[Matrix], hp) -> int:
+    return int(_lib().muon_step_host_grad_workspace_size(_descs(mats), len(mats), ctypes.byref(hp[0])))
+
+
+def muon_step_batched_host_grad(mats: Sequence[Matrix], hp, workspace, stream=None):
+    """muon_step_batched with every G a pinned CPU tensor: the library streams the gradients
+    in chunk by chunk, overlapping the copies with the step of earlier chunks."""
+    for m in mats:
+        if m.G.is_cuda or not m.G.is_pinned():
+            raise ValueError("G must be a pinned CPU tensor (tensor.pin_memory())")
+    st = _lib().muon_step_batched_host_grad(_descs(mats), len(mats), ctypes.byref(hp[0]), workspace.data_ptr(),
+                                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "muon_step_batched_host_grad")
 
 
 def ns_workspace_size(batch: int, rows: int, cols: int, schedule: Schedule) -> int:

@@ -9,6 +9,8 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <functional>
+#include <mutex>
 
 #include "runtime.cuh"
 
@@ -381,6 +383,78 @@ StepLayout plan_step_layout(const muon_matrix_desc* descs, int count, const muon
     return L;
 }
 
+// ---------------------------------------------------------------- host gradients
+// Chunks of a host-gradient step: [begin, end) index ranges of about equal gradient bytes.
+std::vector<std::pair<int, int>> host_grad_chunks(const muon_matrix_desc* d, int count) {
+    std::vector<size_t> bytes(count);
+    size_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        bytes[i] = static_cast<size_t>(d[i].rows) * d[i].cols * (d[i].g_dtype == MUON_F32 ? 4 : 2);
+        total += bytes[i];
+    }
+    const int target = std::min(count, MUON_HOST_GRAD_CHUNKS);
+    std::vector<std::pair<int, int>> chunks;
+    size_t acc = 0;
+    int begin = 0;
+    for (int i = 0; i < count; ++i) {
+        acc += bytes[i];
+        const size_t bound = total / target * (chunks.size() + 1);
+        const int left_items = count - 1 - i, left_chunks = target - static_cast<int>(chunks.size()) - 1;
+        if (i == count - 1 || (acc >= bound && left_items >= left_chunks) || left_items < left_chunks) {
+            chunks.push_back({begin, i + 1});
+            begin = i + 1;
+        }
+    }
+    return chunks;
+}
+
+size_t grad_slot_bytes(const muon_matrix_desc* d, int begin, int end) {
+    size_t b = 0;
+    for (int i = begin; i < end; ++i)
+        b += align_up(static_cast<size_t>(d[i].rows) * d[i].cols * (d[i].g_dtype == MUON_F32 ? 4 : 2), kAlign);
+    return b;
+}
+
+// Workspace of a host-gradient step: the call's status header, then two step workspaces and
+// two gradient staging slots; chunk c uses step workspace and slot c % 2, so the copy stream
+// can fill chunk c + 1's slot and plan tables while chunk c computes.
+struct HostGradLayout {
+    std::vector<std::pair<int, int>> chunks;
+    size_t step_ws = 0;     // one chunk step workspace (largest chunk)
+    size_t slot = 0;        // one staging slot
+    size_t total = 0;
+};
+
+HostGradLayout host_grad_layout(const muon_matrix_desc* d, int count, const muon_hyper* hp) {
+    HostGradLayout L;
+    L.chunks = host_grad_chunks(d, count);
+    for (const auto& c : L.chunks) {
+        std::vector<muon_matrix_desc> sub(d + c.first, d + c.second);
+        for (auto& x : sub) x.G = x.W;   // placement only: the size depends on shapes and dtypes
+        L.step_ws = std::max(L.step_ws, align_up(muon_step_workspace_size(sub.data(), static_cast<int>(sub.size()), hp), kAlign));
+        L.slot = std::max(L.slot, grad_slot_bytes(d, c.first, c.second));
+    }
+    L.total = kHeaderBytes + 2 * L.step_ws + 2 * L.slot;
+    return L;
+}
+
+__global__ void status_or_kernel(unsigned* dst, const unsigned* src) { atomicOr(dst, *src); }
+
+muon_status step_batched(const muon_matrix_desc* descs, int count, const muon_hyper* hp, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream, cudaStream_t upload_stream,
+                         const std::function<muon_status()>& before_launch);
+
+cudaStream_t copy_stream_for_device() {
+    static std::mutex mu;
+    static cudaStream_t streams[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
+}
+
 }  // namespace
 }  // namespace muon
 
@@ -423,12 +497,21 @@ size_t muon_step_workspace_min(const muon_matrix_desc* descs, int count, const m
 
 muon_status muon_step_batched(const muon_matrix_desc* descs, int count, const muon_hyper* hp, void* workspace,
                               size_t ws_bytes, void* stream_) {
+    return step_batched(descs, count, hp, workspace, ws_bytes, static_cast<cudaStream_t>(stream_), nullptr, nullptr);
+}
+
+}  // extern "C"
+
+namespace muon {
+namespace {
+muon_status step_batched(const muon_matrix_desc* descs, int count, const muon_hyper* hp, void* workspace,
+                         size_t ws_bytes, cudaStream_t stream, cudaStream_t upload_stream,
+                         const std::function<muon_status()>& before_launch) {
     muon_status st = check_step_args(descs, count, hp);
     if (st != MUON_OK) return st;
     if (workspace == nullptr) return MUON_ERR_INVALID_ARG;
     if (!aligned256(workspace)) return MUON_ERR_ALIGNMENT;
     if (ws_bytes < muon_step_workspace_min(descs, count, hp)) return MUON_ERR_WORKSPACE_TOO_SMALL;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     const muon_hyper H = *hp;
     const std::vector<float> coeffs(hp->ns.coeffs, hp->ns.coeffs + 3 * hp->ns.n_iters);
     const std::vector<muon_matrix_desc> D(descs, descs + count);
@@ -520,7 +603,87 @@ muon_status muon_step_batched(const muon_matrix_desc* descs, int count, const mu
         if (img.bytes.size() > L.table_bound) return MUON_ERR_WORKSPACE_TOO_SMALL;
         return MUON_OK;
     };
-    return run_plan(kw.k, workspace, L.table_offset, build, stream);
+    return run_plan(kw.k, workspace, L.table_offset, build, stream, upload_stream, before_launch);
+}
+}  // namespace
+}  // namespace muon
+
+extern "C" {
+
+size_t muon_step_host_grad_workspace_size(const muon_matrix_desc* descs, int count, const muon_hyper* hp) {
+    if (check_step_args(descs, count, hp) != MUON_OK) return 0;
+    return host_grad_layout(descs, count, hp).total;
+}
+
+muon_status muon_step_batched_host_grad(const muon_matrix_desc* descs, int count, const muon_hyper* hp,
+                                        void* workspace, size_t ws_bytes, void* stream_) {
+    muon_status st = check_step_args(descs, count, hp);
+    if (st != MUON_OK) return st;
+    if (workspace == nullptr) return MUON_ERR_INVALID_ARG;
+    if (!aligned256(workspace)) return MUON_ERR_ALIGNMENT;
+    for (int i = 0; i < count; ++i) {
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, descs[i].G) != cudaSuccess || a.type != cudaMemoryTypeHost) {
+            cudaGetLastError();
+            return MUON_ERR_INVALID_ARG;
+        }
+    }
+    const HostGradLayout L = host_grad_layout(descs, count, hp);
+    if (ws_bytes < L.total) return MUON_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    cudaStream_t cs = copy_stream_for_device();
+    if (cs == nullptr) return MUON_ERR_CUDA;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    unsigned* status = static_cast<unsigned*>(workspace);
+    uint8_t* step_ws[2] = {ws + kHeaderBytes, ws + kHeaderBytes + L.step_ws};
+    uint8_t* slots[2] = {ws + kHeaderBytes + 2 * L.step_ws, ws + kHeaderBytes + 2 * L.step_ws + L.slot};
+
+    const int nc = static_cast<int>(L.chunks.size());
+    std::vector<cudaEvent_t> ev(static_cast<size_t>(2 * nc + 1), nullptr);
+    auto fail = [&](muon_status s) {
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+        return s;
+    };
+    for (auto& e : ev)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return fail(MUON_ERR_CUDA);
+    // the copy stream joins `stream`'s order (and its capture, if any) here
+    if (cudaMemsetAsync(status, 0, sizeof(unsigned), stream) != cudaSuccess ||
+        cudaEventRecord(ev[0], stream) != cudaSuccess || cudaStreamWaitEvent(cs, ev[0], 0) != cudaSuccess)
+        return fail(MUON_ERR_CUDA);
+    for (int c = 0; c < nc; ++c) {
+        cudaEvent_t copied = ev[1 + 2 * c], done = ev[2 + 2 * c];
+        const int b = L.chunks[c].first, e = L.chunks[c].second;
+        // step workspace and slot c % 2 are free once chunk c - 2 has finished on `stream`
+        if (c >= 2 && cudaStreamWaitEvent(cs, ev[2 + 2 * (c - 2)], 0) != cudaSuccess) return fail(MUON_ERR_CUDA);
+        std::vector<muon_matrix_desc> sub(descs + b, descs + e);
+        std::vector<const void*> src(sub.size());
+        size_t off = 0;
+        for (size_t i = 0; i < sub.size(); ++i) {
+            src[i] = sub[i].G;
+            sub[i].G = slots[c & 1] + off;
+            off += align_up(static_cast<size_t>(sub[i].rows) * sub[i].cols * (sub[i].g_dtype == MUON_F32 ? 4 : 2), kAlign);
+        }
+        // on the copy stream: the chunk's plan tables (inside step_batched), then its
+        // gradients; `stream` waits for both before the chunk's first launch
+        auto copy_in = [&]() -> muon_status {
+            for (size_t i = 0; i < sub.size(); ++i) {
+                const size_t bytes = static_cast<size_t>(sub[i].rows) * sub[i].cols * (sub[i].g_dtype == MUON_F32 ? 4 : 2);
+                if (cudaMemcpyAsync(const_cast<void*>(sub[i].G), src[i], bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+                    return MUON_ERR_CUDA;
+            }
+            if (cudaEventRecord(copied, cs) != cudaSuccess || cudaStreamWaitEvent(stream, copied, 0) != cudaSuccess)
+                return MUON_ERR_CUDA;
+            return MUON_OK;
+        };
+        st = step_batched(sub.data(), static_cast<int>(sub.size()), hp, step_ws[c & 1], L.step_ws, stream, cs, copy_in);
+        if (st != MUON_OK) return fail(st);
+        status_or_kernel<<<1, 1, 0, stream>>>(status, reinterpret_cast<const unsigned*>(step_ws[c & 1]));
+        if (cudaGetLastError() != cudaSuccess || cudaEventRecord(done, stream) != cudaSuccess)
+            return fail(MUON_ERR_CUDA);
+    }
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);   // released once their work completes
+    return MUON_OK;
 }
 
 size_t ns_workspace_size(int batch, int rows, int cols, const muon_ns_schedule* sch) {

@@ -60,7 +60,8 @@ int device_sm_count() {
 }
 
 muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t table_offset,
-                     const std::function<muon_status(Plan&, TableImage&)>& build, cudaStream_t stream) {
+                     const std::function<muon_status(Plan&, TableImage&)>& build, cudaStream_t stream,
+                     cudaStream_t upload_stream, const std::function<muon_status()>& before_launch) {
     std::lock_guard<std::mutex> lk(g_mu);
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
@@ -101,11 +102,16 @@ muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t
         plan = g_plans.back().get();
     }
 
-    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned), stream);
+    cudaStream_t up = upload_stream ? upload_stream : stream;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned), up);
     if (e != cudaSuccess) return MUON_ERR_CUDA;
     if (plan->table_bytes) {
-        e = cudaMemcpyAsync(plan->dev_tables, plan->pinned, plan->table_bytes, cudaMemcpyHostToDevice, stream);
+        e = cudaMemcpyAsync(plan->dev_tables, plan->pinned, plan->table_bytes, cudaMemcpyHostToDevice, up);
         if (e != cudaSuccess) return MUON_ERR_CUDA;
+    }
+    if (before_launch) {
+        const muon_status st = before_launch();
+        if (st != MUON_OK) return st;
     }
     for (const PlanStep& s : plan->steps) {
         if (g_timing.enabled) {

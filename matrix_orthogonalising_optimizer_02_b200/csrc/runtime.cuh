@@ -82,9 +82,14 @@ struct KeyWriter {
 };
 
 // Finds a cached plan for `key` or builds one with `build` (which fills steps and the table
-// image); then copies the tables and runs the steps on `stream`.
+// image); then clears the workspace status word, copies the tables and runs the steps on
+// `stream`.  With an `upload_stream` the status clear and the table copy go there instead,
+// and `before_launch` (if set) runs after they are enqueued and before the first launch:
+// it must order `stream` after the upload (an event).
 muon_status run_plan(const std::vector<uint8_t>& key, void* workspace, size_t table_offset,
-                     const std::function<muon_status(Plan&, TableImage&)>& build, cudaStream_t stream);
+                     const std::function<muon_status(Plan&, TableImage&)>& build, cudaStream_t stream,
+                     cudaStream_t upload_stream = nullptr,
+                     const std::function<muon_status()>& before_launch = nullptr);
 
 // Tensor map of a row-major bf16 matrix (rows x cols, pitch = cols) with a box of 64 columns
 // x box_rows rows, 128-byte swizzle, zero fill out of bounds.

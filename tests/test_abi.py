@@ -134,3 +134,18 @@ def test_timing_api_is_host_only():
         assert ms == 0 and n == 0 and work == 0
     with pytest.raises(mb.MuonError):
         mb._check(mb.load().muon_timing_read(99, None, None, None), "timing_read")
+
+
+def test_host_gradient_workspace_is_host_only_and_bounded():
+    lib = mb.load()
+    hp, _keep = mb.hyper(0.02)
+    shapes = [(4096, 4096)] * 4 + [(4096, 11008)] * 2 + [(11008, 4096)]
+    d = _descs(shapes * 4)
+    n = len(shapes) * 4
+    full = lib.muon_step_workspace_size(d, n, ctypes.byref(hp))
+    host = lib.muon_step_host_grad_workspace_size(d, n, ctypes.byref(hp))
+    # one chunk's step workspace plus two staging slots: well below the whole set's workspace
+    # plus its gradients, and at least two slots of the largest chunk's bf16 gradients
+    grads = sum(r * c * 2 for r, c in shapes * 4)
+    assert 2 * grads / 8 <= host < full
+    assert lib.muon_step_host_grad_workspace_size(d, 0, ctypes.byref(hp)) == 0
