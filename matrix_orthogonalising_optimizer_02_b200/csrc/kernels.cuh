@@ -62,7 +62,7 @@ inline void tc_set_segments(TcProblem& P, int na, int nb, int max_order) {
         }
 }
 
-constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64, kTcStages = 3;   // pair (2-CTA) tile
+constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64, kTcStages = 4;   // pair (2-CTA) tile
 constexpr int kTcThreads = 384;            // 4 role warps + 8 epilogue warps
 constexpr int kTcEpilogueThreads = 256;
 // Tile code: problem (12 bits) | m block (10 bits) | n block (10 bits).

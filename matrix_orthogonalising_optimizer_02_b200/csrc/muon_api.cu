@@ -384,7 +384,9 @@ StepLayout plan_step_layout(const muon_matrix_desc* descs, int count, const muon
 }
 
 // ---------------------------------------------------------------- host gradients
-// Chunks of a host-gradient step: [begin, end) index ranges of about equal gradient bytes.
+// Chunks of a host-gradient step: [begin, end) index ranges.  Chunk boundaries fall at
+// (j + 1/2) / target of the gradient bytes, so the first chunk -- whose copy nothing can
+// hide -- carries half a share and the last one and a half.
 std::vector<std::pair<int, int>> host_grad_chunks(const muon_matrix_desc* d, int count) {
     std::vector<size_t> bytes(count);
     size_t total = 0;
@@ -398,9 +400,10 @@ std::vector<std::pair<int, int>> host_grad_chunks(const muon_matrix_desc* d, int
     int begin = 0;
     for (int i = 0; i < count; ++i) {
         acc += bytes[i];
-        const size_t bound = total / target * (chunks.size() + 1);
+        const size_t bound = static_cast<size_t>(static_cast<double>(total) * (chunks.size() + 0.5) / target);
         const int left_items = count - 1 - i, left_chunks = target - static_cast<int>(chunks.size()) - 1;
-        if (i == count - 1 || (acc >= bound && left_items >= left_chunks) || left_items < left_chunks) {
+        const bool may_close = static_cast<int>(chunks.size()) + 1 < target;   // the last chunk takes the rest
+        if (i == count - 1 || (may_close && ((acc >= bound && left_items >= left_chunks) || left_items < left_chunks))) {
             chunks.push_back({begin, i + 1});
             begin = i + 1;
         }
