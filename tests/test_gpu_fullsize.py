@@ -92,3 +92,109 @@ def test_low_rank_batch_full(sched, nsplit):
     Yf = Y.float()
     s = torch.linalg.svdvals(Yf)
     assert torch.isfinite(s).all() and float(s.max()) < 1.6
+
+
+@pytest.mark.parametrize("rows,cols", [(4096, 11008), (11008, 4096)])
+def test_rank_one_input_maps_to_phi5_at_full_size(rows, cols):
+    """A rank-1 input has one singular value, exactly 1 after the Frobenius pre-scale, so
+    Newton-Schulz returns phi_5(1) u v^T: a closed form that holds at any size.  u and v have
+    entries +-2^e, so u v^T is exact in bf16 and every later stage (Gram, polynomial, apply,
+    each rounded to bf16 and accumulated in fp32) treats all entries alike up to a power of
+    two: the device result stays exactly rank-1 and only its scalar carries rounding.  (A
+    generic bf16-rounded u v^T is not rank-1: its rounding noise has tiny singular values,
+    which the iteration lifts by design.)  phi_5(1) is the oracle's own iteration on 1 x 1."""
+    r = workloads.rng(1201)
+    u = np.where(r.random(rows) < 0.5, -1.0, 1.0) * 2.0 ** r.integers(-2, 3, rows)
+    v = np.where(r.random(cols) < 0.5, -1.0, 1.0) * 2.0 ** r.integers(-2, 3, cols)
+    X = torch.outer(torch.tensor(u, dtype=torch.float32), torch.tensor(v, dtype=torch.float32))
+    X = X.to(torch.bfloat16).cuda().contiguous()
+    Y = torch.empty_like(X)
+    sch = mb.Schedule.fixed(5)
+    ws = mb.workspace(mb.ns_workspace_size(1, rows, cols, sch))
+    mb.ns_orthogonalize(X, Y, sch, ws)
+    assert mb.device_status(ws) == mb.MUON_OK
+    phi = float(orc.newton_schulz(np.ones((1, 1)), orc.fixed_schedule(5))[0, 0])
+    assert abs(phi - 0.69644) < 1e-4
+    uh = u / np.linalg.norm(u)
+    vh = v / np.linalg.norm(v)
+    Yh = host(Y)
+    # project onto u v^T and measure what is left, without forming another full matrix
+    coef = float(uh @ Yh @ vh)
+    resid2 = float(np.sum(Yh * Yh)) - coef * coef
+    assert abs(coef - phi) <= 2e-2 * phi
+    assert np.sqrt(max(resid2, 0.0)) <= 1e-3 * phi
+
+
+def test_zero_gradient_from_zero_momentum_is_pure_decay():
+    """M = 0 and G = 0 give X0 = 0, a zero Newton-Schulz output (0 / (0 + eps)), and the
+    update reduces to W1 = bf16((1 - lr wd) W0) on every matrix of a mixed set."""
+    shapes = [(4096, 4096), (4096, 11008), (11008, 4096), (136, 264), (264, 136)]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1202)
+    mats = []
+    for rows, cols in shapes:
+        W = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda").normal_(0.0, 0.02, generator=gen)
+        G = torch.zeros((rows, cols), dtype=torch.bfloat16, device="cuda")
+        M = torch.zeros((rows, cols), dtype=torch.float32, device="cuda")
+        mats.append(mb.Matrix(W, G, M, torch.empty_like(W)))
+    before = [host(m.W) for m in mats]
+    hp = mb.hyper(lr=LR, beta=BETA, weight_decay=WD)
+    ws = mb.workspace(mb.muon_step_workspace_size(mats, hp))
+    mb.muon_step_batched(mats, hp, ws)
+    assert mb.device_status(ws) == mb.MUON_OK
+    decay = np.float32(1.0) - np.float32(LR) * np.float32(WD)
+    for m, W0 in zip(mats, before):
+        assert not torch.any(m.M) and not torch.any(m.O_out.float())
+        want = orc.round_to_bf16((np.float32(W0) * decay).astype(np.float64))
+        assert np.array_equal(host(m.W), want)
+
+
+def test_muon_cayley_full_size_tall_and_wide():
+    """MuonCayley at the 16 x 4096 x 1024 Stiefel workload size, and its wide transpose
+    (16 x 1024 x 4096): two steps each, one sampled matrix against the oracle, the manifold
+    invariant on every matrix."""
+    for wide in (False, True):
+        batch, n, k, lr, beta = 16, 4096, 1024, 3e-3, 0.9
+        Ws = workloads.stiefel_problem(seed=1203, batch=batch, n=n, k=k)
+        if wide:
+            Ws = np.ascontiguousarray(np.swapaxes(Ws, 1, 2))
+        W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+        M = torch.zeros_like(W)
+        rows, cols = W.shape[1], W.shape[2]
+        ws = mb.workspace(mb.muon_cayley_workspace_size(batch, rows, cols))
+        i = 5
+        Wr, Mr = host(W[i]), np.zeros((rows, cols))
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(1204)
+        G = torch.empty_like(W)
+        for _ in range(2):
+            workloads.device_normal_(G, 1.0, gen)
+            Gi = host(G[i])
+            mb.muon_cayley_step(W, G, M, lr, beta, ws, center=True)
+            Wr, Mr = orc.muon_cayley_step(Wr, Gi, Mr, lr, float(np.float32(beta)))
+        assert mb.device_status(ws) == mb.MUON_OK
+        assert np.max(np.abs(host(W[i]) - Wr)) <= 2e-5
+        Wd = W.double()
+        gram = Wd @ Wd.transpose(1, 2) if wide else Wd.transpose(1, 2) @ Wd
+        eye = torch.eye(gram.shape[-1], dtype=torch.float64, device="cuda")
+        assert float((gram - eye).abs().max()) <= 1e-5
+        del W, M, G, ws, Wd, gram
+        torch.cuda.empty_cache()
+
+
+def test_host_gradient_step_matches_device_step_on_eight_llama_layers():
+    """The host-gradient path at scale: 8 Llama-7B layers (56 matrices, 3.2 GB of bf16
+    gradients, 8 chunks) give bit-identical W and M to the device-resident step."""
+    layer = [(4096, 4096)] * 4 + [(4096, 11008)] * 2 + [(11008, 4096)]
+    shapes = layer * 8
+    dev_set = _device_set(shapes, 1205, ())
+    host_set = [mb.Matrix(m.W.clone(), m.G.cpu().pin_memory(), m.M.clone()) for m in dev_set]
+    hp = mb.hyper(lr=LR, beta=BETA, weight_decay=WD)
+    ws_d = mb.workspace(mb.muon_step_workspace_size(dev_set, hp))
+    ws_h = mb.workspace(mb.muon_step_host_grad_workspace_size(host_set, hp))
+    for _ in range(2):
+        mb.muon_step_batched(dev_set, hp, ws_d)
+        mb.muon_step_batched_host_grad(host_set, hp, ws_h)
+    assert mb.device_status(ws_d) == mb.MUON_OK and mb.device_status(ws_h) == mb.MUON_OK
+    for d, h in zip(dev_set, host_set):
+        assert torch.equal(d.W, h.W) and torch.equal(d.M, h.M)
