@@ -62,7 +62,10 @@ inline void tc_set_segments(TcProblem& P, int na, int nb, int max_order) {
         }
 }
 
-constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64, kTcStages = 4;   // pair (2-CTA) tile
+constexpr int kTcBM = 256, kTcBN = 256, kTcBK = 64;   // pair (2-CTA) tile
+// Depth of the TMA ring.  On the power-capped part 4 stages measured fastest: a deeper ring
+// keeps the tensor pipe busier per cycle but lowers the sustained clock by more.
+constexpr int kTcStages = 4;
 constexpr int kTcThreads = 384;            // 4 role warps + 8 epilogue warps
 constexpr int kTcEpilogueThreads = 256;
 // Tile code: problem (12 bits) | m block (10 bits) | n block (10 bits).

@@ -614,9 +614,9 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
                   long long aug_stride, unsigned* d_status) {
     auto Ai = [&](int i) { return Aug + i * aug_stride; };
     std::vector<SimtProblem> pr;
-    // Gaussian elimination with partial pivoting on [C | y], fp64, two levels: 128-column
+    // Gaussian elimination with partial pivoting on [C | y], fp64, two levels: kLuBlock-wide
     // block columns factorised with nb-wide panels (updates confined to the block column),
-    // then one row-swap + unit-lower solve over the trailing columns and one K = 128
+    // then one row-swap + unit-lower solve over the trailing columns and one K = kLuBlock
     // trailing update per block column.
     const int nb = lu_panel_width(N);
     for (int J0 = 0; J0 < N; J0 += kLuBlock) {

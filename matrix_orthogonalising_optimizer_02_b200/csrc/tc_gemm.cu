@@ -7,7 +7,7 @@
 // and its 128 columns of B, so every SM reads half of B's bytes a 1-SM 128 x 256 tile
 // would; each CTA's TMEM holds its 128 rows x 256 fp32 columns, twice (double buffer).
 // Roles per CTA (384 threads):
-//   warp 0 lane 0 : TMA producer -- 6-stage ring of (128 x 64 A, 128 x 64 B) bf16 tiles,
+//   warp 0 lane 0 : TMA producer -- kTcStages-deep ring of (128 x 64 A, 128 x 64 B) bf16 tiles,
 //                   128-byte swizzled, K-major or MN-major per problem; the loads of both
 //                   CTAs count on the leader CTA's "full" barrier (.cta_group::2 form)
 //   warp 1 lane 0 : MMA issuer (leader CTA only) -- commits free the stage in both CTAs
