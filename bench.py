@@ -257,9 +257,18 @@ def _stiefel(gen):
     kinds = {k: mb.timing_read(k) for k in ("tc_f32", "simt_gemm", "lu", "misc")}
     work = kinds["tc_f32"][2] + kinds["simt_gemm"][2] + kinds["lu"][2]
     ms = _time_ms(lambda: mb.stiefel_cayley_step(W, G, 1e-2, ws), 1, 3)
+    # ALU roofline of the fp32 SIMT products: 148 SMs x 128 fp32 lanes x 2 FLOP per FMA at
+    # the maximum SM clock (1965 MHz) = 74.4 TFLOP/s
+    simt_ms, _, simt_work = kinds["simt_gemm"]
+    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    simt_tflops = simt_work / max(simt_ms * 1e-3, 1e-12) / 1e12
     out["stiefel_16x4096x1024_step"] = {"ms": ms, "fma_tflops": work / (ms * 1e-3) / 1e12,
                                         "kernel_ms": {k: v[0] for k, v in kinds.items()},
-                                        "tc_f32_tflops": kinds["tc_f32"][2] / max(kinds["tc_f32"][0] * 1e-3, 1e-12) / 1e12}
+                                        "tc_f32_tflops": kinds["tc_f32"][2] / max(kinds["tc_f32"][0] * 1e-3, 1e-12) / 1e12,
+                                        "roofline": {"bound": "alu", "kernel": "simt_gemm_kernel (fp32 and fp64 FMA)",
+                                                     "achieved": simt_tflops, "peak": fp32_peak, "unit": "TFLOP/s",
+                                                     "frac": simt_tflops / fp32_peak,
+                                                     "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"}}
     return out
 
 
