@@ -231,6 +231,10 @@ MUON_API muon_status muon_timing_reset(void);
 MUON_API muon_status muon_timing_read(int kind, double* ms, long long* launches, double* work);
 
 MUON_API const char* muon_status_string(muon_status s);
+/* Description of the last MUON_ERR_CUDA failure on the calling thread: the library call
+ * that failed (a launch names its index and kernel kind) and the CUDA error name and text;
+ * "" if none.  The string stays valid until the thread's next failing call. */
+MUON_API const char* muon_last_error(void);
 MUON_API const char* muon_build_info(void);
 
 #ifdef __cplusplus

@@ -32,7 +32,7 @@ EXPORTED = (
     "muon_workspace_device_status", "muon_timing_enable", "muon_timing_reset", "muon_timing_read",
     "muon_status_string", "muon_build_info", "muon_frobenius_prescale_static",
     "muon_cayley_workspace_size", "muon_cayley_step", "muon_step_host_grad_workspace_size",
-    "muon_step_batched_host_grad",
+    "muon_step_batched_host_grad", "muon_last_error",
 )
 
 
@@ -40,6 +40,10 @@ class MuonError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         msg = _lib().muon_status_string(status).decode() if _LIB is not None else str(status)
+        if status == MUON_ERR_CUDA and _LIB is not None:
+            detail = _LIB.muon_last_error()
+            if detail:
+                msg += f": {detail.decode()}"
         super().__init__(f"{where}: {msg} (status {status})")
 
 
@@ -86,6 +90,7 @@ def _lib():
         "muon_timing_reset": (c_int, []),
         "muon_timing_read": (c_int, [c_int, POINTER(c_double), POINTER(c_longlong), POINTER(c_double)]),
         "muon_status_string": (ctypes.c_char_p, [c_int]),
+        "muon_last_error": (ctypes.c_char_p, []),
         "muon_build_info": (ctypes.c_char_p, []),
         "muon_cayley_workspace_size": (c_size_t, [c_int, c_int, c_int]),
         "muon_cayley_step": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_float, c_float, c_int,

@@ -44,13 +44,23 @@ void drain_timing_locked() {
 
 Plan::~Plan() {
     if (last_use) {
-        cudaEventSynchronize(last_use);
+        if (recorded) cudaEventSynchronize(last_use);   // the last table copy has finished
         cudaEventDestroy(last_use);
     }
     if (pinned) cudaFreeHost(pinned);
+    cudaGetLastError();   // leave no error of this cleanup pending for the caller's next check
 }
 
-muon_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MUON_OK : MUON_ERR_CUDA; }
+namespace {
+thread_local char g_last_error[256] = "";
+}
+
+muon_status cuda_error(cudaError_t e, const char* where) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+    return MUON_ERR_CUDA;
+}
+
+muon_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MUON_OK : cuda_error(e, "CUDA call"); }
 
 int device_sm_count() {
     int dev = 0, sms = 148;
@@ -64,7 +74,12 @@ muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t
                      cudaStream_t upload_stream, const std::function<muon_status()>& before_launch) {
     std::lock_guard<std::mutex> lk(g_mu);
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_error(e, "cudaGetDevice");
+    // An error left pending by earlier, unrelated work would otherwise be reported by the
+    // first launch check below as this call's own failure: clear it, and name it if this call
+    // then fails.
+    const cudaError_t pending = cudaGetLastError();
     KeyWriter kw;
     kw.put_bytes(key_in.data(), key_in.size());
     kw.put(dev);
@@ -91,29 +106,52 @@ muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t
         p->table_bytes = img.bytes.size();
         p->dev_tables = img.dev_base;
         if (p->table_bytes) {
-            if (cudaHostAlloc(reinterpret_cast<void**>(&p->pinned), p->table_bytes, cudaHostAllocDefault) !=
-                cudaSuccess)
-                return MUON_ERR_CUDA;
+            e = cudaHostAlloc(reinterpret_cast<void**>(&p->pinned), p->table_bytes, cudaHostAllocDefault);
+            if (e != cudaSuccess) return cuda_error(e, "cudaHostAlloc of the plan tables");
             std::memcpy(p->pinned, img.bytes.data(), p->table_bytes);
         }
-        if (cudaEventCreateWithFlags(&p->last_use, cudaEventDisableTiming) != cudaSuccess) return MUON_ERR_CUDA;
-        if (g_plans.size() >= kMaxPlans) g_plans.erase(g_plans.begin());
+        e = cudaEventCreateWithFlags(&p->last_use, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_error(e, "cudaEventCreate");
+        if (g_plans.size() >= kMaxPlans) {   // evict the least recently used plan no graph holds
+            for (size_t i = 0; i < g_plans.size(); ++i) {
+                if (!g_plans[i]->captured) {
+                    g_plans.erase(g_plans.begin() + static_cast<long>(i));
+                    break;
+                }
+            }
+        }
         g_plans.push_back(std::move(p));
         plan = g_plans.back().get();
     }
 
+    auto fail = [&](cudaError_t err, const char* where) {
+        char buf[160];
+        if (pending != cudaSuccess)
+            std::snprintf(buf, sizeof(buf), "%s (an earlier %s was pending on entry)", where, cudaGetErrorName(pending));
+        else
+            std::snprintf(buf, sizeof(buf), "%s", where);
+        return cuda_error(err, buf);
+    };
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return fail(e, "cudaStreamIsCapturing");
+    const bool capturing = cap != cudaStreamCaptureStatusNone;
+    if (capturing) plan->captured = true;
     cudaStream_t up = upload_stream ? upload_stream : stream;
-    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(unsigned), up);
-    if (e != cudaSuccess) return MUON_ERR_CUDA;
+    e = cudaMemsetAsync(workspace, 0, sizeof(unsigned), up);
+    if (e != cudaSuccess) return fail(e, "status clear");
     if (plan->table_bytes) {
         e = cudaMemcpyAsync(plan->dev_tables, plan->pinned, plan->table_bytes, cudaMemcpyHostToDevice, up);
-        if (e != cudaSuccess) return MUON_ERR_CUDA;
+        if (e != cudaSuccess) return fail(e, "table upload");
     }
     if (before_launch) {
         const muon_status st = before_launch();
         if (st != MUON_OK) return st;
     }
-    for (const PlanStep& s : plan->steps) {
+    static const char* const kind_names[MUON_KERNEL_KINDS] = {"momentum", "scale", "ns_gemm", "update",
+                                                              "simt_gemm", "lu", "misc", "tc_f32"};
+    for (size_t si = 0; si < plan->steps.size(); ++si) {
+        const PlanStep& s = plan->steps[si];
         if (g_timing.enabled) {
             TimingRec r{s.kind, s.work, nullptr, nullptr};
             cudaEventCreate(&r.e0);
@@ -125,10 +163,24 @@ muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t
         } else {
             e = s.run(stream);
         }
-        if (e != cudaSuccess) return MUON_ERR_CUDA;
+        if (e != cudaSuccess) {
+            char buf[96];
+            std::snprintf(buf, sizeof(buf), "launch %zu of %zu (%s)", si, plan->steps.size(),
+                          s.kind >= 0 && s.kind < MUON_KERNEL_KINDS ? kind_names[s.kind] : "?");
+            return fail(e, buf);
+        }
     }
-    e = cudaEventRecord(plan->last_use, stream);
-    return from_cuda(e);
+    if (!capturing) {
+        e = cudaEventRecord(plan->last_use, stream);
+        if (e != cudaSuccess) return fail(e, "cudaEventRecord");
+        plan->recorded = true;
+    }
+    return MUON_OK;
+}
+
+void TmapPool::note_failure(const void* base, int rows, int cols, int box) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed for %p (%d x %d bf16, box %d)",
+                  base, rows, cols, box);
 }
 
 bool encode_bf16_tmap(CUtensorMap* out, const void* base, int rows, int cols, int box_rows) {
@@ -157,6 +209,8 @@ bool encode_bf16_tmap(CUtensorMap* out, const void* base, int rows, int cols, in
 }  // namespace muon
 
 extern "C" {
+
+const char* muon_last_error(void) { return muon::g_last_error; }
 
 muon_status muon_timing_enable(int enable) {
     std::lock_guard<std::mutex> lk(muon::g_mu);

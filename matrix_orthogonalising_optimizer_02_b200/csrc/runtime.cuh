@@ -63,7 +63,11 @@ struct Plan {
     size_t table_bytes = 0;
     uint8_t* dev_tables = nullptr;   // destination in the workspace
     std::vector<PlanStep> steps;
-    cudaEvent_t last_use = nullptr;
+    cudaEvent_t last_use = nullptr;   // recorded after each run outside stream capture
+    bool recorded = false;
+    // Run at least once under stream capture: a graph may hold a copy node that reads
+    // `pinned`, so the plan is never evicted.
+    bool captured = false;
     ~Plan();
 };
 
@@ -106,12 +110,17 @@ struct TmapPool {
     std::vector<Entry> entries;
     bool failed = false;
     explicit TmapPool(TableImage& i) : img(i) {}
+    // Records the first failed encoding as the thread's last library error.
+    void note_failure(const void* base, int rows, int cols, int box);
     const CUtensorMap* get(const void* base, int rows, int cols, int box) {
         if (base == nullptr) return nullptr;
         for (auto& e : entries)
             if (e.base == base && e.rows == rows && e.cols == cols && e.box == box) return img.dev<CUtensorMap>(e.off);
         CUtensorMap tm;
-        if (!encode_bf16_tmap(&tm, base, rows, cols, box)) failed = true;
+        if (!encode_bf16_tmap(&tm, base, rows, cols, box)) {
+            if (!failed) note_failure(base, rows, cols, box);
+            failed = true;
+        }
         const size_t off = img.add(&tm, sizeof(tm), 128);
         entries.push_back({base, rows, cols, box, off});
         return img.dev<CUtensorMap>(off);
@@ -120,5 +129,8 @@ struct TmapPool {
 
 int device_sm_count();
 muon_status from_cuda(cudaError_t e);
+// Records `where` and the CUDA error as the calling thread's last library error (read with
+// muon_last_error) and returns MUON_ERR_CUDA.
+muon_status cuda_error(cudaError_t e, const char* where);
 
 }  // namespace muon

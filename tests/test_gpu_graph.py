@@ -41,3 +41,37 @@ def test_step_graph_replay_matches_eager():
     torch.cuda.synchronize()
     for a, b in zip(eager, graphed):
         assert torch.equal(a.W, b.W) and torch.equal(a.M, b.M)
+
+
+def test_captured_plan_survives_plan_cache_churn():
+    """A captured graph's table copy reads the plan's pinned host tables, so a plan used under
+    capture must outlive any number of later plans: replaying after 40 other plans (more than
+    the cache holds) still equals the eager steps, and no call reports an error."""
+    eager, graphed = _set(91), _set(91)
+    hp = mb.hyper(lr=0.02, weight_decay=0.1)
+    ws_e = mb.workspace(mb.muon_step_workspace_size(eager, hp))
+    ws_g = mb.workspace(mb.muon_step_workspace_size(graphed, hp))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        mb.muon_step_batched(graphed, hp, ws_g, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    mb.muon_step_batched(eager, hp, ws_e)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        mb.muon_step_batched(graphed, hp, ws_g)
+    # 40 distinct plans: ns_orthogonalize over 40 shapes
+    sch = mb.Schedule.fixed(1)
+    for i in range(40):
+        rows, cols = 64 + 8 * i, 96
+        X = torch.ones((rows, cols), dtype=torch.bfloat16, device="cuda")
+        Y = torch.empty_like(X)
+        ws = mb.workspace(mb.ns_workspace_size(1, rows, cols, sch))
+        mb.ns_orthogonalize(X, Y, sch, ws)
+        assert mb.device_status(ws) == mb.MUON_OK
+    for _ in range(2):
+        g.replay()
+        mb.muon_step_batched(eager, hp, ws_e)
+    torch.cuda.synchronize()
+    for a, b in zip(eager, graphed):
+        assert torch.equal(a.W, b.W) and torch.equal(a.M, b.M)
