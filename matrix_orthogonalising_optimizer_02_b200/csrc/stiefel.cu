@@ -626,10 +626,17 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
             const size_t smem = static_cast<size_t>(panel_pitch(N - j0)) * w * sizeof(double);
             const double lu_flops = 2.0 * (N - j0) * w * w * B;
             plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
-                static bool attr = false;
-                if (!attr) {
-                    cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
-                    attr = true;
+                // the function attribute is per device: set once on each (launches run under
+                // the plan cache's lock)
+                static bool attr_set[64] = {};
+                int dev = 0;
+                cudaError_t e = cudaGetDevice(&dev);
+                if (e != cudaSuccess) return e;
+                if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+                if (!attr_set[dev]) {
+                    e = cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
+                    if (e != cudaSuccess) return e;
+                    attr_set[dev] = true;
                 }
                 lu_panel_kernel<<<B, 1024, smem, s>>>(Aug, ld, aug_stride, N, j0, w, piv, N, d_status);
                 return cudaGetLastError();

@@ -393,7 +393,15 @@ size_t tc_gemm_smem_bytes() { return SMEM_TOTAL; }
 cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, int num_tiles, unsigned* d_status,
                            int num_sms, cudaStream_t stream) {
     if (num_tiles <= 0) return cudaSuccess;
-    static int max_pairs = 0;
+    // Function attributes and the cluster occupancy are per device: set up once on each.
+    // (Launches run under the plan cache's lock, so this needs none of its own.)
+    constexpr int kMaxDevices = 64;
+    static int max_pairs_of[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t de = cudaGetDevice(&dev);
+    if (de != cudaSuccess) return de;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int& max_pairs = max_pairs_of[dev];
     if (max_pairs == 0) {
         cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
         if (e != cudaSuccess) return e;
@@ -410,7 +418,10 @@ cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, in
         cfg.numAttrs = 1;
         int clusters = 0;
         e = cudaOccupancyMaxActiveClusters(&clusters, tc_gemm_kernel, &cfg);
-        if (e != cudaSuccess || clusters <= 0) clusters = num_sms / 2;
+        if (e != cudaSuccess || clusters <= 0) {
+            cudaGetLastError();   // fall back to one pair per two SMs; leave no error pending
+            clusters = num_sms / 2;
+        }
         max_pairs = clusters;
     }
     const int pairs = num_tiles < max_pairs ? num_tiles : max_pairs;
