@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "runtime.cuh"
+#include "simt_async.cuh"
 
 namespace muon {
 namespace {
@@ -294,8 +295,11 @@ muon_status build_ns_simt(Plan& plan, TableImage& img, std::vector<NsMat>& mats,
             const SimtProblem* dp = img.dev<SimtProblem>(po);
             const uint32_t* dt = img.dev<uint32_t>(to);
             const int nt = static_cast<int>(tiles.size());
+            bool a_kc = false;
+            const bool async = simt_async_suits(probs, &a_kc);
             plan.steps.push_back({MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t st) {
-                                      return simt_gemm_launch(dp, dt, nt, st);
+                                      return async ? simt_gemm_async_launch(dp, dt, nt, st, a_kc)
+                                                   : simt_gemm_launch(dp, dt, nt, st);
                                   }});
         }
     }

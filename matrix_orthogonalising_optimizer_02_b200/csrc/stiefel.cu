@@ -17,6 +17,7 @@
 #include <cmath>
 
 #include "runtime.cuh"
+#include "simt_async.cuh"
 
 namespace muon {
 namespace {
@@ -529,8 +530,11 @@ void add_gemm(Plan& plan, TableImage& img, const std::vector<SimtProblem>& all, 
         const SimtProblem* dp = img.dev<SimtProblem>(img.add(probs.data(), probs.size() * sizeof(SimtProblem), kAlign));
         const uint32_t* dt = img.dev<uint32_t>(img.add(tiles.data(), tiles.size() * sizeof(uint32_t), kAlign));
         const int nt = static_cast<int>(tiles.size());
+        bool a_kc = false;
+        const bool async = !f64_acc && simt_async_suits(probs, &a_kc);
         plan.steps.push_back({MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t s) {
-                                  return simt_gemm_launch(dp, dt, nt, s, f64_acc);
+                                  return async ? simt_gemm_async_launch(dp, dt, nt, s, a_kc)
+                                               : simt_gemm_launch(dp, dt, nt, s, f64_acc);
                               }});
     }
 }
