@@ -181,6 +181,31 @@ __global__ void split3_kernel(const Split3Item* __restrict__ items, int count) {
     it.dst[2 * n + e] = __float2bfloat16_rn(r2);
 }
 
+// fp32 copy of a k x k block of an fp64 matrix (the same round-to-nearest the SIMT GEMM
+// applies when it loads an fp64 operand), so the product that reads it can take the fp32
+// multi-stage GEMM.
+struct BlockCastItem {
+    const double* src;
+    float* dst;           // rows x cols, contiguous
+    long long ld;         // source row pitch
+    long long block0;
+    int rows, cols;
+};
+__global__ void block_cast_kernel(const BlockCastItem* __restrict__ items, int count) {
+    const long long b = blockIdx.x;
+    int lo = 0, hi = count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (items[mid].block0 <= b) lo = mid; else hi = mid - 1;
+    }
+    const BlockCastItem& it = items[lo];
+    const long long n = static_cast<long long>(it.rows) * it.cols;
+    const long long e = (b - it.block0) * blockDim.x + threadIdx.x;
+    if (e >= n) return;
+    const long long r = e / it.cols, c = e % it.cols;
+    it.dst[e] = static_cast<float>(it.src[r * it.ld + c]);
+}
+
 // Panel factorisation (partial pivoting) of rows j0..N-1, columns j0..j0+nb-1, held in
 // shared memory column by column with an odd pitch (consecutive rows in consecutive words,
 // so the per-row sweeps are free of bank conflicts).  Records the pivot row of each column
@@ -505,7 +530,8 @@ size_t stiefel_tables_bound(int batch, int n, int k) {
     const size_t tmaps = static_cast<size_t>(batch) * 3 * 3 * 2 * (sizeof(CUtensorMap) + 128);
     const size_t prob_bytes = std::max(sizeof(SimtProblem), sizeof(TcProblem)) + 16;
     size_t b = static_cast<size_t>(t) * batch * sizeof(uint32_t) + static_cast<size_t>(probs) * batch * prob_bytes +
-               static_cast<size_t>(probs) * 2 * kAlign + tmaps + static_cast<size_t>(batch) * 16 * 64 + 64 * kAlign;
+               static_cast<size_t>(probs) * 2 * kAlign + tmaps + static_cast<size_t>(batch) * 16 * 64 + 64 * kAlign +
+               static_cast<size_t>(batch) * 4 * sizeof(BlockCastItem) + 2 * kAlign;   // fp32 block copies
     return align_up(b + 4096, kAlign);
 }
 
@@ -830,6 +856,25 @@ void add_tc_splitk(Plan& plan, TableImage& img, const std::vector<TcProblem>& pr
                           }});
 }
 
+void add_block_cast(Plan& plan, TableImage& img, const std::vector<BlockCastItem>& in) {
+    std::vector<BlockCastItem> items(in);
+    long long block0 = 0;
+    double bytes = 0;
+    for (auto& it : items) {
+        it.block0 = block0;
+        const long long n = static_cast<long long>(it.rows) * it.cols;
+        block0 += (n + 255) / 256;
+        bytes += 12.0 * n;
+    }
+    const BlockCastItem* di = img.dev<BlockCastItem>(img.add(items.data(), items.size() * sizeof(BlockCastItem), kAlign));
+    const int ni = static_cast<int>(items.size());
+    const long long nb = block0;
+    plan.steps.push_back({MUON_KERNEL_MISC, bytes, [=](cudaStream_t s) {
+                              block_cast_kernel<<<static_cast<unsigned>(nb), 256, 0, s>>>(di, ni);
+                              return cudaGetLastError();
+                          }});
+}
+
 void add_split3(Plan& plan, TableImage& img, const std::vector<Split3Item>& in) {
     std::vector<Split3Item> items(in);
     long long block0 = 0;
@@ -954,10 +999,22 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
         aug_neg_transpose_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
         return cudaGetLastError();
     }});
+    // fp32 copies of two k x k blocks of each augmented matrix (into the split-K scratch, free
+    // between the reductions), as the B operands of the n x k products that follow
+    auto blocks32 = [&](int i, int which) { return part + (2LL * i + which) * kk; };
+    auto cast_blocks = [&](long long off0, long long off1) {
+        std::vector<BlockCastItem> items;
+        for (int i = 0; i < B; ++i)
+            for (int which = 0; which < 2; ++which)
+                items.push_back({Ai(i) + (which == 0 ? off0 : off1), blocks32(i, which), ld, 0, k, k});
+        add_block_cast(plan, img, items);
+    };
+    auto Bm32 = [&](int i, int which) { return Mat{blocks32(i, which), k, false, false}; };
     // b = W - V (cQ) - W (-c P^T)
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, k), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
+    cast_blocks(k, k * ld + k);
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Bm32(i, 0), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
     add_gemm(plan, img, pr); pr.clear();
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + k), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Bm32(i, 1), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
     add_gemm(plan, img, pr); pr.clear();
     // C = I + c B U
     plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * N * B, [=](cudaStream_t s) {
@@ -972,9 +1029,10 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
     add_gemm_splitk(plan, img, pr, part); pr.clear();
     add_lu_solve(plan, img, Aug, piv, N, ncols, k, B, ld, aug_stride, d_status);
     // W_new = b - c V z_top - c W z_bot, then copy into W
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Am(i, N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
+    cast_blocks(N, k * ld + N);
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Bm32(i, 0), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
     add_gemm(plan, img, pr); pr.clear();
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Am(i, k * ld + N), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Bm32(i, 1), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
     add_gemm(plan, img, pr); pr.clear();
     const size_t bytes = static_cast<size_t>(nk) * B * sizeof(float);
     plan.steps.push_back({MUON_KERNEL_MISC, 2.0 * bytes, [=](cudaStream_t s) {
