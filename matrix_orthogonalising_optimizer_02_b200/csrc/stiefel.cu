@@ -364,15 +364,15 @@ __device__ __forceinline__ void apply_swaps(double* a, long long ld, const int* 
 }
 
 // Row swaps then unit-lower solve U12 = L11^-1 A12 with the w x w triangle at (r0, r0), for
-// the columns [c_lo, ncols) -- (128 / G) columns per block of 128 threads.  The group's
-// first lane applies the swaps; every lane of a warp reaches the shuffles.
+// the columns [c_lo, ncols) -- blockDim.x / G columns per block.  The group's first lane
+// applies the swaps; every lane of a warp reaches the shuffles.
 template <int R, int G>
 __device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const int* pv, int r0, int w, int c_lo,
                                                 int ncols, double* T) {
     constexpr int P = R + 2;
     load_block_cols<R, P>(T, a, ld, r0, w);
     __syncthreads();
-    const int c = c_lo + static_cast<int>(blockIdx.x) * (128 / G) + static_cast<int>(threadIdx.x) / G;
+    const int c = c_lo + static_cast<int>(blockIdx.x * (blockDim.x / G) + threadIdx.x / G);
     const int h = static_cast<int>(threadIdx.x) % G;
     const bool live = c < ncols;
     if (live && h == 0) apply_swaps(a, ld, pv, r0, w, c);
@@ -416,28 +416,33 @@ __global__ void lu_swap_cols_kernel(double* Aug, long long ld, long long stride,
 
 // After a block column J0..J0+JB-1 is factorised: for every column c >= c_lo, apply the
 // block's JB row swaps in order, then solve with the JB x JB unit-lower L11 (U12 = L11^-1 A12).
-constexpr int kLuBlock = 64, kLuLanes = 4;
-__global__ void __launch_bounds__(128)
+// The 128 x 128 triangle (133 KB) is in dynamic shared memory, shared by the block's 64
+// columns (512 threads, 8 lanes per column).
+constexpr int kLuBlock = 128, kLuLanes = 8, kTrsmThreads = 512;
+constexpr size_t kLuTriangleBytes = static_cast<size_t>(kLuBlock) * (kLuBlock + 2) * sizeof(double);
+__global__ void __launch_bounds__(kTrsmThreads)
 lu_block_swap_trsm_kernel(double* Aug, long long ld, long long stride, int J0, int JB, int c_lo, int ncols,
                           const int* piv, long long piv_stride) {
-    __shared__ __align__(16) double T[kLuBlock * (kLuBlock + 2)];
+    extern __shared__ __align__(16) double T[];
     swap_trsm_block<kLuBlock, kLuLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, J0, JB, c_lo,
                                         ncols, T);
 }
 
 // Back substitution on one diagonal block: rows i0..i0+bs-1 of the right-hand columns
-// (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows); 32 columns per block.
-constexpr int kBackBlock = 64, kBackLanes = 4, kBackPitch = kBackBlock + 2;
-__global__ void __launch_bounds__(128)
+// (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows); 64 columns per block of 512
+// threads, the triangle and the reciprocals of its diagonal in dynamic shared memory.
+constexpr int kBackBlock = 128, kBackLanes = 8, kBackPitch = kBackBlock + 2;
+constexpr size_t kBackSmemBytes = (static_cast<size_t>(kBackBlock) * kBackPitch + kBackBlock) * sizeof(double);
+__global__ void __launch_bounds__(kTrsmThreads)
 back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, int rhs0, int nrhs) {
-    __shared__ __align__(16) double T[kBackBlock * kBackPitch];
-    __shared__ double dinv[kBackBlock];
+    extern __shared__ __align__(16) double T[];
+    double* dinv = T + kBackBlock * kBackPitch;
     double* a = Aug + blockIdx.y * stride;
     load_block_cols<kBackBlock, kBackPitch>(T, a, ld, i0, bs);
     for (int l = threadIdx.x; l < kBackBlock; l += blockDim.x)
         dinv[l] = l < bs ? 1.0 / a[(i0 + static_cast<long long>(l)) * ld + i0 + l] : 0.0;
     __syncthreads();
-    const int c = static_cast<int>(blockIdx.x) * (128 / kBackLanes) + static_cast<int>(threadIdx.x) / kBackLanes;
+    const int c = static_cast<int>(blockIdx.x * (blockDim.x / kBackLanes) + threadIdx.x / kBackLanes);
     const int h = static_cast<int>(threadIdx.x) % kBackLanes;
     const bool live = c < nrhs;
     double* col = a + rhs0 + (live ? c : 0) + i0 * ld;
@@ -638,6 +643,23 @@ SimtProblem gemm(Mat A, Mat B, void* out, long long ldo, bool o64, const void* E
     return P;
 }
 
+// Allows `kernel` `bytes` of dynamic shared memory on the current device (once per device;
+// launches run under the plan cache's lock).
+template <auto Kernel>
+cudaError_t big_smem(size_t bytes) {
+    static bool set_on[64] = {};   // one flag set per kernel (template argument)
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!set_on[dev]) {
+        e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+        if (e != cudaSuccess) return e;
+        set_on[dev] = true;
+    }
+    return cudaSuccess;
+}
+
 // Gaussian elimination with partial pivoting on the augmented fp64 systems [C | y]
 // (N x ncols, row pitch ld, batch B), then back substitution: z overwrites y.
 void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int ncols, int k, int B, long long ld,
@@ -701,9 +723,11 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
         if (right > 0) {
             const int c_lo = J0 + JB;
             plan.steps.push_back({MUON_KERNEL_LU, 1.0 * JB * JB * right * B, [=](cudaStream_t s) {
-                constexpr int cols_per_block = 128 / kLuLanes;
-                lu_block_swap_trsm_kernel<<<dim3((right + cols_per_block - 1) / cols_per_block, B), 128, 0, s>>>(
-                    Aug, ld, aug_stride, J0, JB, c_lo, ncols, piv, N);
+                constexpr int cols_per_block = kTrsmThreads / kLuLanes;
+                cudaError_t e = big_smem<lu_block_swap_trsm_kernel>(kLuTriangleBytes);
+                if (e != cudaSuccess) return e;
+                lu_block_swap_trsm_kernel<<<dim3((right + cols_per_block - 1) / cols_per_block, B), kTrsmThreads,
+                                            kLuTriangleBytes, s>>>(Aug, ld, aug_stride, J0, JB, c_lo, ncols, piv, N);
                 return cudaGetLastError();
             }});
             if (N - J0 - JB > 0) {
@@ -722,9 +746,11 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
     for (int q = nblk - 1; q >= 0; --q) {
         const int i0 = q * kBackBlock, bs = std::min(kBackBlock, N - i0);
         plan.steps.push_back({MUON_KERNEL_LU, 1.0 * bs * bs * k * B, [=](cudaStream_t s) {
-            constexpr int cols_per_block = 128 / kBackLanes;
-            back_diag_kernel<<<dim3((k + cols_per_block - 1) / cols_per_block, B), 128, 0, s>>>(Aug, ld, aug_stride, i0,
-                                                                                               bs, N, k);
+            constexpr int cols_per_block = kTrsmThreads / kBackLanes;
+            cudaError_t e = big_smem<back_diag_kernel>(kBackSmemBytes);
+            if (e != cudaSuccess) return e;
+            back_diag_kernel<<<dim3((k + cols_per_block - 1) / cols_per_block, B), kTrsmThreads, kBackSmemBytes, s>>>(
+                Aug, ld, aug_stride, i0, bs, N, k);
             return cudaGetLastError();
         }});
         if (i0 > 0) {
