@@ -79,25 +79,26 @@ def oracle_sample(iters):
     return time.perf_counter() - t0, ns_flops_algorithmic(4096, 4096, iters)
 
 
-def recorded_traffic():
-    """DRAM bytes per NS GEMM launch from the committed ncu summary, if it was captured on
-    the kernel sources as they are now (else None)."""
+def recorded_traffic(layers_per_launch):
+    """DRAM bytes per NS GEMM launch: the committed ncu summary's per-launch bytes on one
+    layer (7 independent matrices, so traffic grows in proportion) times the layers one launch
+    covers, if the summary was captured on the kernel sources as they are now (else None)."""
     import hashlib
     md = os.path.join(ROOT, "profiles", "tc_gemm_llama7b_1layer.md")
     if not os.path.exists(md):
         return None
     fields = {}
     for line in open(md):
-        if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch_full_set",
+        if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch_one_layer",
                                                            "kernel_source_sha256_16"):
             k, v = line.split(":", 1)
             fields[k.strip()] = v.strip()
     h = hashlib.sha256()
     for f in ("tc_gemm.cu", "kernels.cuh", "ptx_sm100.cuh"):
         h.update(open(os.path.join(ROOT, "matrix_orthogonalising_optimizer_02_b200", "csrc", f), "rb").read())
-    if fields.get("kernel_source_sha256_16") != h.hexdigest()[:16] or LAYERS != 32:
+    if fields.get("kernel_source_sha256_16") != h.hexdigest()[:16] or "traffic_bytes_per_launch_one_layer" not in fields:
         return None
-    return int(fields["traffic_bytes_per_launch_full_set"])
+    return int(int(fields["traffic_bytes_per_launch_one_layer"]) * layers_per_launch)
 
 
 def set_flops():
@@ -466,8 +467,9 @@ def main():
         "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel (NS Gram/polynomial/apply)",
                      "achieved": ns_tflops, "peak": tf_sust, "unit": "TFLOP/s", "frac": ns_tflops / tf_sust,
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-                     "work_per_launch": ns_flops / max(ns_launches, 1), "traffic": recorded_traffic(),
-                     "traffic_unit": "bytes per launch (ncu dram__bytes_read+write, one layer scaled x32)"},
+                     "work_per_launch": ns_flops / max(ns_launches, 1),
+                     "traffic": recorded_traffic(LAYERS * 15 * n_prof / max(ns_launches, 1)),
+                     "traffic_unit": "bytes per launch (ncu dram__bytes_read+write on one layer, scaled by the layers one launch covers)"},
         "e2e": {"value": e2e_ms / world, "unit": "ms", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4},
         "clocks": clk,
         "total_ns_flops_per_set": total_flops,

@@ -116,8 +116,11 @@ typedef struct {
 } muon_hyper;
 
 /* Bytes of workspace muon_step_batched needs for this set (0 if the arguments are
- * invalid).  The set is processed in one pass when ws_bytes is at least this size; a
- * smaller workspace of at least muon_step_workspace_min() is processed in groups. */
+ * invalid).  The step runs the set in consecutive groups whose Newton-Schulz buffers share
+ * one region of at most 5 GiB (one group if the whole set fits; a single larger matrix
+ * forms its own group); this size covers that region.  A smaller workspace of at least
+ * muon_step_workspace_min() is processed in smaller groups.  Grouping does not change any
+ * result: every matrix goes through the same arithmetic. */
 MUON_API size_t muon_step_workspace_size(const muon_matrix_desc* descs, int count, const muon_hyper* hp);
 MUON_API size_t muon_step_workspace_min(const muon_matrix_desc* descs, int count, const muon_hyper* hp);
 

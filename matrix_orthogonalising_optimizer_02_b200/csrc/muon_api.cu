@@ -8,6 +8,7 @@
 // iterate -> transpose back because B is symmetric.
 #include <algorithm>
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <functional>
 #include <mutex>
@@ -366,10 +367,18 @@ muon_status check_step_args(const muon_matrix_desc* descs, int count, const muon
     return MUON_OK;
 }
 
+// Largest Newton-Schulz data region (X ping-pong, A, B, partial sums) of one group of a step;
+// a set needing more runs as consecutive groups that reuse one region.  On the Llama-7B-shaped
+// set (40 GB of such data) one group per step took 511 ms, 4 groups 478, 8 groups 460, 16
+// groups 463 and 32 groups 468 ms on the same part (groups of about 5 GB are the 8-group
+// case), and the step's workspace shrinks from the whole set's data to one group's.
+constexpr size_t kStepGroupBytes = static_cast<size_t>(5) << 30;
+
 StepLayout plan_step_layout(const muon_matrix_desc* descs, int count, const muon_hyper* hp, size_t ws_bytes) {
     StepLayout L;
     L.table_bound = step_tables_bound(descs, count, hp->ns);
-    const size_t budget = ws_bytes > kHeaderBytes + L.table_bound ? ws_bytes - kHeaderBytes - L.table_bound : 0;
+    const size_t room = ws_bytes > kHeaderBytes + L.table_bound ? ws_bytes - kHeaderBytes - L.table_bound : 0;
+    const size_t budget = std::min(room, kStepGroupBytes);
     std::vector<int> cur;
     for (int i = 0; i < count; ++i) {
         std::vector<int> trial = cur;
@@ -489,10 +498,8 @@ const char* muon_build_info(void) {
 
 size_t muon_step_workspace_size(const muon_matrix_desc* descs, int count, const muon_hyper* hp) {
     if (check_step_args(descs, count, hp) != MUON_OK) return 0;
-    std::vector<int> all(count);
-    for (int i = 0; i < count; ++i) all[i] = i;
-    return kHeaderBytes + align_up(group_data_bytes(descs, all, hp->ns), kAlign) +
-           step_tables_bound(descs, count, hp->ns);
+    const StepLayout L = plan_step_layout(descs, count, hp, SIZE_MAX);
+    return L.table_offset + L.table_bound;
 }
 
 size_t muon_step_workspace_min(const muon_matrix_desc* descs, int count, const muon_hyper* hp) {
