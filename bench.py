@@ -79,6 +79,13 @@ def oracle_sample(iters):
     return time.perf_counter() - t0, ns_flops_algorithmic(4096, 4096, iters)
 
 
+def workload_config(shapes):
+    """The `config` object both arms print for the parameter set `shapes`."""
+    return {"workload": WORKLOAD if LAYERS == 32 else f"{WORKLOAD}_{LAYERS}layer", "matrices": len(shapes),
+            "params": sum(r * c for r, c in shapes), "ns_iters": 5, "coeffs": list(KJ), "lr": LR, "beta": BETA,
+            "weight_decay": WD, "scale": "moonlight", "l2": "inputs (52 GB) larger than L2; no flush"}
+
+
 def recorded_traffic(layers_per_launch):
     """DRAM bytes per NS GEMM launch: the committed ncu summary's per-launch bytes on one
     layer (7 independent matrices, so traffic grows in proportion) times the layers one launch
@@ -304,7 +311,7 @@ def run_reference(args, rank, world):
     out = {"metric": "Muon full-step ms per param set (Llama-7B-shaped set)", "value": ms, "unit": "ms",
            "impl": "reference", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-           "data": "synthetic", "config": {"workload": WORKLOAD, "matrices": 224, "params": 6476005376},
+           "data": "synthetic", "config": workload_config(set_shapes()),
            "cpu_baseline": {"value": ms, "unit": "ms", "cores": cpu_cores(), "kind": "oracle", "sample": sample},
            "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -452,9 +459,7 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded on-device normal draws, Llama-7B shapes)",
-        "config": {"workload": WORKLOAD if LAYERS == 32 else f"{WORKLOAD}_{LAYERS}layer", "matrices": len(shapes), "params": sum(r * c for r, c in shapes),
-                   "ns_iters": 5, "coeffs": list(KJ), "lr": LR, "beta": BETA, "weight_decay": WD,
-                   "scale": "moonlight", "l2": "inputs (52 GB) larger than L2; no flush"},
+        "config": workload_config(shapes),
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "matrices_per_s": len(shapes) * world / (ms_step * 1e-3),
         "ns_tflops": ns_tflops,
