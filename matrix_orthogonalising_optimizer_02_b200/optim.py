@@ -26,14 +26,17 @@ def _check_matrix(p):
 
 
 class _Workspaces:
+    """One workspace per device, grown to the largest request: the library's calls are
+    ordered on the current stream, so successive calls can share it."""
+
     def __init__(self):
         self.bufs = {}
 
-    def get(self, key, nbytes, device):
-        ws = self.bufs.get(key)
-        if ws is None or ws.numel() < nbytes or ws.device != device:
+    def get(self, nbytes, device):
+        ws = self.bufs.get(device)
+        if ws is None or ws.numel() < nbytes:
             ws = mb.workspace(nbytes, device=device)
-            self.bufs[key] = ws
+            self.bufs[device] = ws
         return ws
 
 
@@ -59,7 +62,7 @@ class Muon(torch.optim.Optimizer):
         if closure is not None:
             with torch.enable_grad():
                 loss = closure()
-        for gi, group in enumerate(self.param_groups):
+        for group in self.param_groups:
             mats = []
             for p in group["params"]:
                 if p.grad is None:
@@ -75,7 +78,7 @@ class Muon(torch.optim.Optimizer):
                               eps=group["eps"])
             hp = mb.hyper(group["lr"], group["momentum"], group["weight_decay"], group["nesterov"],
                           group["scale_mode"], sch)
-            ws = self._ws.get(gi, mb.muon_step_workspace_size(mats, hp), mats[0].W.device)
+            ws = self._ws.get(mb.muon_step_workspace_size(mats, hp), mats[0].W.device)
             mb.muon_step_batched(mats, hp, ws)
         return loss
 
@@ -101,15 +104,15 @@ class MuonCayley(torch.optim.Optimizer):
         if closure is not None:
             with torch.enable_grad():
                 loss = closure()
-        for gi, group in enumerate(self.param_groups):
-            for pi, p in enumerate(group["params"]):
+        for group in self.param_groups:
+            for p in group["params"]:
                 if p.grad is None:
                     continue
                 state = self.state[p]
                 if "momentum_buffer" not in state:
                     state["momentum_buffer"] = torch.zeros_like(p)
                 n, k = p.shape
-                ws = self._ws.get((gi, pi), mb.muon_cayley_workspace_size(1, n, k), p.device)
+                ws = self._ws.get(mb.muon_cayley_workspace_size(1, n, k), p.device)
                 mb.muon_cayley_step(p.data, p.grad.contiguous(), state["momentum_buffer"], group["lr"],
                                     group["momentum"], ws, center=group["center"])
         return loss
