@@ -149,3 +149,31 @@ def test_host_gradient_workspace_is_host_only_and_bounded():
     grads = sum(r * c * 2 for r, c in shapes * 4)
     assert 2 * grads / 8 <= host < full
     assert lib.muon_step_host_grad_workspace_size(d, 0, ctypes.byref(hp)) == 0
+
+
+def test_host_gradient_step_argument_errors_are_host_side():
+    """Validation of the host-gradient step happens before any CUDA call."""
+    lib = mb.load()
+    hp, _keep = mb.hyper(0.02)
+    ws = ctypes.c_void_p(1 << 24)
+    d = _descs([(64, 64)])
+    assert lib.muon_step_batched_host_grad(None, 1, ctypes.byref(hp), ws, 1 << 30, None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_step_batched_host_grad(d, 0, ctypes.byref(hp), ws, 1 << 30, None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_step_batched_host_grad(d, 1, ctypes.byref(hp), None, 1 << 30, None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_step_batched_host_grad(d, 1, ctypes.byref(hp), ctypes.c_void_p((1 << 24) + 16), 1 << 30,
+                                           None) == mb.MUON_ERR_ALIGNMENT
+    d = _descs([(60, 64)])
+    assert lib.muon_step_batched_host_grad(d, 1, ctypes.byref(hp), ws, 1 << 30, None) == \
+        mb.MUON_ERR_UNSUPPORTED_SHAPE
+
+
+def test_last_error_is_a_string_and_grouping_bounds_the_step_workspace():
+    lib = mb.load()
+    assert isinstance(lib.muon_last_error(), bytes)
+    hp, _keep = mb.hyper(0.02)
+    layer = [(4096, 4096)] * 4 + [(4096, 11008)] * 2 + [(11008, 4096)]
+    d = _descs(layer * 32)
+    full = lib.muon_step_workspace_size(d, len(layer) * 32, ctypes.byref(hp))
+    # the 224-matrix set runs in groups whose NS buffers share at most 5 GiB
+    per_layer = sum(2 * r * c * 2 + 2 * min(r, c) ** 2 * 2 for r, c in layer)
+    assert 4 * per_layer < full < (5 << 30) + (64 << 20)
