@@ -214,9 +214,18 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
                         for (int mb = 0; mb < mbs; ++mb)
                             if (kTcBN * nb + kTcBN - 1 >= kTcBM * mb) tiles.push_back(tile_code(p, mb, nb));
                 } else {
+                    // Neighbouring CTA pairs (consecutive tiles) share one block of X and sweep
+                    // the r x r polynomial B, which stays in L2: down the columns for a wide X
+                    // (B X), along the rows for a tall X (X B).  The other order streams a tall
+                    // X from DRAM once per column block.
                     const int mbs = (m.rows + kTcBM - 1) / kTcBM, nbs = (m.cols + kTcBN - 1) / kTcBN;
-                    for (int nb = 0; nb < nbs; ++nb)
-                        for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(p, mb, nb));
+                    if (!m.tall) {
+                        for (int nb = 0; nb < nbs; ++nb)
+                            for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(p, mb, nb));
+                    } else {
+                        for (int mb = 0; mb < mbs; ++mb)
+                            for (int nb = 0; nb < nbs; ++nb) tiles.push_back(tile_code(p, mb, nb));
+                    }
                 }
             }
             if (pool.failed) return MUON_ERR_CUDA;
