@@ -368,3 +368,26 @@ def test_muon_cayley_step_on_a_wide_parameter_keeps_rows_orthonormal():
     # the same gradient without centring does move W
     W2, _ = orc.muon_cayley_step(W, G_rows, np.zeros((rows, cols)), lr=0.5, beta=0.0, center=False)
     assert np.max(np.abs(W2 - W)) > 1e-3
+
+
+@pytest.mark.parametrize("rows,cols", [(24, 40), (40, 24)])
+def test_full_step_on_a_rank_one_gradient_has_a_closed_form(rows, cols):
+    """beta = 0 and M0 = 0 make M1 = G.  With G = u v^T on entries +-2^e, the bf16 cast is exact and
+    G has one singular value, so the Frobenius pre-scale makes it 1 and Newton-Schulz returns
+    phi_5(1) u^ v^T (u^, v^ unit vectors), whatever the orientation.  The step is then
+    W1 = (1 - lr wd) W0 - lr * 0.2 sqrt(max(rows, cols)) * phi_5(1) u^ v^T.  This pins the whole
+    chain (momentum, cast, pre-scale, iteration, transpose handling, scale, decay order) at
+    once; phi_5(1) = 0.69644 is the rank-1 worked value."""
+    r = workloads.rng(57)
+    u = np.where(r.random(rows) < 0.5, -1.0, 1.0) * 2.0 ** r.integers(-3, 3, rows)
+    v = np.where(r.random(cols) < 0.5, -1.0, 1.0) * 2.0 ** r.integers(-3, 3, cols)
+    G = np.outer(u, v) * 2.0 ** -10
+    assert np.array_equal(orc.round_to_bf16(G), G)
+    W0 = orc.round_to_bf16(r.standard_normal((rows, cols)) * 0.02)
+    lr, wd = 0.02, 0.1
+    out = orc.muon_step(W0, G, np.zeros((rows, cols)), lr=lr, beta=0.0, weight_decay=wd)
+    phi = 0.69644
+    uh, vh = u / np.linalg.norm(u), v / np.linalg.norm(v)
+    assert np.allclose(out["O"], phi * np.outer(uh, vh), atol=1e-5)
+    want = (1 - lr * wd) * W0 - lr * 0.2 * np.sqrt(max(rows, cols)) * phi * np.outer(uh, vh)
+    assert np.max(np.abs(out["W1_exact"] - want)) < 1e-6
