@@ -20,7 +20,8 @@
  *    evaluated in the rank-2k Woodbury form of §6.2 (a 2k x 2k solve plus n x k GEMMs).
  *
  * Conventions shared by every entry point:
- *  - All matrices are dense row-major.  Matrix pointers are DEVICE pointers; descriptor
+ *  - All matrices are dense row-major.  Matrix pointers are DEVICE pointers (except the
+ *    gradients of muon_step_batched_host_grad, which sit in pinned host memory); descriptor
  *    arrays, schedules and coefficient tables are HOST pointers read during the call only.
  *  - The caller owns every buffer, including the workspace; the library never allocates
  *    device memory.  The workspace holds the library's tables between calls: a call with
@@ -30,8 +31,9 @@
  *    asynchronous on `stream` and never synchronises it, except
  *    muon_workspace_device_status(), which does.
  *  - Host-side argument checks run before any launch; on error nothing is launched and
- *    buffers are untouched.  Launch failures return MUON_ERR_CUDA.  Device-side
- *    conditions (a non-finite Frobenius norm, a kernel wait that ran out of time) are
+ *    buffers are untouched.  Launch failures return MUON_ERR_CUDA (muon_last_error() then
+ *    names the failing call).  Device-side conditions (a non-finite Frobenius norm, a zero
+ *    or non-finite pivot in the Cayley solve, a kernel wait that ran out of time) are
  *    recorded in the workspace and read back by muon_workspace_device_status().
  *  - bf16 matrices handled on the tensor-core path need rows % 8 == 0, cols % 8 == 0 and
  *    16-byte aligned pointers (TMA and 128-bit accesses); fp32 mode has no shape limit
@@ -132,7 +134,8 @@ MUON_API muon_status muon_step_batched(const muon_matrix_desc* descs, int count,
 
 /* The same step with every G in pinned (page-locked) host memory; W, M and O_out stay on
  * the device.  The set is cut, in descriptor order, into up to MUON_HOST_GRAD_CHUNKS
- * chunks of about equal gradient bytes.  The chunks' gradients are copied into two staging
+ * chunks of about equal gradient bytes (the first, whose copy nothing can hide, about half
+ * a share).  The chunks' gradients are copied into two staging
  * slots of the workspace on a library-owned copy stream, one cudaMemcpyAsync per matrix,
  * while the previous chunk's step runs on `stream`, so the host-to-device transfer
  * overlaps the computation of earlier chunks.  Results equal those of muon_step_batched on
@@ -158,7 +161,10 @@ MUON_API muon_status ns_orthogonalize(const void* X_in, int in_dtype, void* X_ou
 
 /* Stiefel-manifold step for a contiguous batch of column-orthonormal W (n x k fp32,
  * n >= k): tangent projection of G (n x k fp32), then the Cayley retraction with
- * c = lr/2 in Woodbury form (2k x 2k LU with partial pivoting, fp32, no TF32).
+ * c = lr/2 in Woodbury form.  The direction's two products (W^T G and W sym(.)) run on the
+ * tensor cores as three bf16 planes (fp32-exact operands, fp32 accumulation); every product
+ * that enters the retraction runs in fp32 FMA arithmetic (no TF32); the 2k x 2k system is
+ * solved by fp64 Gaussian elimination with partial pivoting.
  * W is updated in place; G is read.  n < k returns MUON_ERR_UNSUPPORTED_SHAPE (transpose
  * the problem, as the page advises).  k <= 4096. */
 MUON_API size_t stiefel_workspace_size(int batch, int n, int k);
