@@ -165,12 +165,35 @@ class Matrix:
     O_out: Optional[object] = None
 
 
-def _descs(mats: Sequence[Matrix]):
+def _need(t, name: str, cuda: bool = True, device=None):
+    """Checks a tensor handed to the library by its data pointer: dense (a strided view's
+    pointer would be read as another matrix) and on the expected device."""
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (the library reads it as a dense row-major array)")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if cuda and device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _descs(mats: Sequence[Matrix], g_on_host: bool = False):
+    import torch
     arr = (MatrixDesc * len(mats))()
     for i, m in enumerate(mats):
+        if m.W.dim() != 2:
+            raise ValueError("W must be a 2-D matrix")
         rows, cols = m.W.shape
         if tuple(m.G.shape) != (rows, cols) or tuple(m.M.shape) != (rows, cols):
             raise ValueError("W, G and M must have the same 2-D shape")
+        if m.M.dtype != torch.float32:
+            raise TypeError("the momentum buffer M must be fp32")
+        _need(m.W, "W")
+        _need(m.M, "M", device=m.W.device)
+        _need(m.G, "G", cuda=not g_on_host, device=m.W.device)
+        if m.O_out is not None:
+            if tuple(m.O_out.shape) != (rows, cols):
+                raise ValueError("O_out must have W's shape")
+            _need(m.O_out, "O_out", device=m.W.device)
         arr[i] = MatrixDesc(m.W.data_ptr(), m.G.data_ptr(), m.M.data_ptr(),
                             m.O_out.data_ptr() if m.O_out is not None else None,
                             rows, cols, _dtype_code(m.W), _dtype_code(m.G))
@@ -199,7 +222,8 @@ def muon_step_batched(mats: Sequence[Matrix], hp, workspace, stream=None):
 
 
 def muon_step_host_grad_workspace_size(mats: Sequence[Matrix], hp) -> int:
-    return int(_lib().muon_step_host_grad_workspace_size(_descs(mats), len(mats), ctypes.byref(hp[0])))
+    return int(_lib().muon_step_host_grad_workspace_size(_descs(mats, g_on_host=True), len(mats),
+                                                         ctypes.byref(hp[0])))
 
 
 def muon_step_batched_host_grad(mats: Sequence[Matrix], hp, workspace, stream=None):
@@ -208,7 +232,8 @@ def muon_step_batched_host_grad(mats: Sequence[Matrix], hp, workspace, stream=No
     for m in mats:
         if m.G.is_cuda or not m.G.is_pinned():
             raise ValueError("G must be a pinned CPU tensor (tensor.pin_memory())")
-    st = _lib().muon_step_batched_host_grad(_descs(mats), len(mats), ctypes.byref(hp[0]), workspace.data_ptr(),
+    st = _lib().muon_step_batched_host_grad(_descs(mats, g_on_host=True), len(mats), ctypes.byref(hp[0]),
+                                            workspace.data_ptr(),
                                             workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "muon_step_batched_host_grad")
 
@@ -218,6 +243,8 @@ def ns_workspace_size(batch: int, rows: int, cols: int, schedule: Schedule) -> i
 
 
 def ns_orthogonalize(X_in, X_out, schedule: Schedule, workspace, stream=None):
+    _need(X_in, "X_in")
+    _need(X_out, "X_out", device=X_in.device)
     if X_in.dim() == 2:
         batch, (rows, cols) = 1, X_in.shape
     else:
@@ -237,6 +264,8 @@ def stiefel_workspace_size(batch: int, n: int, k: int) -> int:
 
 
 def stiefel_cayley_step(W, G, lr: float, workspace, stream=None):
+    _need(W, "W")
+    _need(G, "G", device=W.device)
     if W.dim() == 2:
         batch, (n, k) = 1, W.shape
     else:
@@ -252,6 +281,8 @@ def frobenius_prescale_static(X_in, X_out, fp32_mode: bool = False, eps: float =
                               stream=None):
     """X_out = X0 / (||X0||_F + eps) per matrix without a workspace: the library's fixed
     internal scratch is used instead (see muon_frobenius_prescale_static in the header)."""
+    _need(X_in, "X_in")
+    _need(X_out, "X_out", device=X_in.device)
     if X_in.dim() == 2:
         batch, (rows, cols) = 1, X_in.shape
     else:
@@ -270,6 +301,9 @@ def muon_cayley_workspace_size(batch: int, n: int, k: int) -> int:
 
 
 def muon_cayley_step(W, G, M, lr: float, beta: float, workspace, center: bool = True, stream=None):
+    _need(W, "W")
+    _need(G, "G", device=W.device)
+    _need(M, "M", device=W.device)
     if W.dim() == 2:
         batch, (n, k) = 1, W.shape
     else:

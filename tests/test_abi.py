@@ -177,3 +177,22 @@ def test_last_error_is_a_string_and_grouping_bounds_the_step_workspace():
     # the 224-matrix set runs in groups whose NS buffers share at most 5 GiB
     per_layer = sum(2 * r * c * 2 + 2 * min(r, c) ** 2 * 2 for r, c in layer)
     assert 4 * per_layer < full < (5 << 30) + (64 << 20)
+
+
+def test_binding_rejects_tensors_it_cannot_pass_by_pointer():
+    """The binding hands the library raw data pointers, so it refuses strided views, a
+    non-fp32 momentum buffer and tensors off the GPU before any library call."""
+    import torch
+    W = torch.zeros((8, 16), dtype=torch.bfloat16)
+    M = torch.zeros((8, 16), dtype=torch.float32)
+    hp = mb.hyper(0.02)
+    with pytest.raises(ValueError, match="contiguous"):
+        mb.muon_step_workspace_size([mb.Matrix(torch.zeros((16, 8), dtype=torch.bfloat16).t(), W, M)], hp)
+    with pytest.raises(TypeError, match="fp32"):
+        mb.muon_step_workspace_size([mb.Matrix(W, W, M.to(torch.bfloat16))], hp)
+    with pytest.raises(ValueError, match="CUDA"):
+        mb.muon_step_workspace_size([mb.Matrix(W, W, M)], hp)
+    with pytest.raises(ValueError, match="contiguous"):
+        mb.ns_orthogonalize(torch.zeros((16, 8)).t(), torch.zeros((8, 16)), mb.Schedule.fixed(1), torch.zeros(1))
+    with pytest.raises(ValueError, match="CUDA"):
+        mb.stiefel_cayley_step(torch.zeros((16, 8)), torch.zeros((16, 8)), 0.01, torch.zeros(1))

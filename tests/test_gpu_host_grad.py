@@ -55,7 +55,7 @@ def test_host_gradient_step_rejects_pageable_gradients():
     host = [mb.Matrix(m.W, m.G.cpu().pin_memory(), m.M) for m in dev]
     ws = mb.workspace(mb.muon_step_host_grad_workspace_size(host, hp))
     pageable = np.zeros(SHAPES[0], dtype=np.uint16)
-    descs = mb._descs(host)
+    descs = mb._descs(host, g_on_host=True)
     descs[0].G = pageable.ctypes.data
     lib = mb.load()
     st = lib.muon_step_batched_host_grad(descs, len(host), ctypes.byref(hp[0]), ws.data_ptr(),
