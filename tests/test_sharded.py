@@ -1,7 +1,7 @@
 """Matrix-ownership sharding: the assignment (host logic) and the owner-computes /
-broadcast exchange with world_size 2 on CPU (gloo).  The stand-in step marks each
-owned matrix with its owner's rank, so after the exchange every rank must hold the
-same weights, each changed exactly once, by its owner."""
+broadcast exchange on CPU (gloo) with world sizes 2 and 4, and within a subgroup.  The
+stand-in step marks each owned matrix with its owner's rank, so after the exchange every
+rank must hold the same weights, each changed exactly once, by its owner."""
 import os
 import socket
 
@@ -36,28 +36,35 @@ def _free_port():
     return port
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, port, q, members=None):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=__import__("datetime").timedelta(seconds=60))
     try:
-        shapes = [(64, 32), (32, 64), (48, 48), (16, 80), (80, 16), (8, 8)]
+        # every rank takes part in creating the subgroup, only its members in the exchange
+        group = dist.new_group(members) if members is not None else None
+        if members is not None and rank not in members:
+            q.put((rank, "ok"))
+            return
+        shapes = [(64, 32), (32, 64), (48, 48), (16, 80), (80, 16), (8, 8), (24, 24), (40, 8)]
         g = torch.Generator().manual_seed(5)
-        weights = [torch.randn(s, generator=g) for s in shapes]     # identical on both ranks
+        weights = [torch.randn(s, generator=g) for s in shapes]     # identical on every rank
         before = [w.clone() for w in weights]
+        my = dist.get_rank(group) if group is not None else rank
 
         def step_owned(indices):
             for i in indices:
-                weights[i].add_(float(rank + 1))
+                weights[i].add_(float(my + 1))
 
-        sh = ShardedMuonStep(weights, step_owned)
+        sh = ShardedMuonStep(weights, step_owned, group=group)
         sh.step()
         for i, w in enumerate(weights):
-            assert torch.equal(w, before[i] + float(sh.owner[i] + 1))
+            assert torch.equal(w, before[i] + float(sh.owner[i] + 1))   # changed once, by its owner
+        size = dist.get_world_size(group)
         sums = torch.tensor([float(sum(w.sum() for w in weights))])
-        gathered = [torch.zeros(1) for _ in range(world)]
-        dist.all_gather(gathered, sums)
-        assert torch.equal(gathered[0], gathered[1])
+        gathered = [torch.zeros(1) for _ in range(size)]
+        dist.all_gather(gathered, sums, group=group)
+        assert all(torch.equal(x, gathered[0]) for x in gathered)
         q.put((rank, "ok"))
     except Exception as e:  # pragma: no cover - reported to the parent
         q.put((rank, repr(e)))
@@ -65,14 +72,25 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_owner_computes_then_broadcast_gloo_world2():
+def _run(world, members=None):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, members)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(timeout=120)
     results = dict(q.get(timeout=5) for _ in procs)
-    assert results == {0: "ok", 1: "ok"}
+    assert results == {r: "ok" for r in range(world)}
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_owner_computes_then_broadcast_gloo(world):
+    _run(world)
+
+
+def test_owner_computes_then_broadcast_within_a_subgroup():
+    """Ranks 1 and 3 of 4 shard among themselves: owners are group ranks, broadcasts use
+    their global ranks."""
+    _run(4, members=[1, 3])
