@@ -244,6 +244,15 @@ MUON_API const char* muon_status_string(muon_status s);
  * that failed (a launch names its index and kernel kind) and the CUDA error name and text;
  * "" if none.  The string stays valid until the thread's next failing call. */
 MUON_API const char* muon_last_error(void);
+
+/* Self-test of the bounded device waits (failure detection): launches one CTA that waits,
+ * through the pipeline's own wait routine, on an mbarrier that nothing completes.  The wait
+ * gives up after its limit (4 s), the kernel records MUON_ERR_DEVICE_TIMEOUT in the
+ * workspace status word and ends; read it with muon_workspace_device_status().  The
+ * context stays usable.  No counterpart on the source pages.
+ * Errors: INVALID_ARG (null workspace or ws_bytes < 256), ALIGNMENT (workspace not
+ * 256-byte aligned), CUDA. */
+MUON_API muon_status muon_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* stream);
 MUON_API const char* muon_build_info(void);
 
 #ifdef __cplusplus

@@ -32,7 +32,7 @@ EXPORTED = (
     "muon_workspace_device_status", "muon_timing_enable", "muon_timing_reset", "muon_timing_read",
     "muon_status_string", "muon_build_info", "muon_frobenius_prescale_static",
     "muon_cayley_workspace_size", "muon_cayley_step", "muon_step_host_grad_workspace_size",
-    "muon_step_batched_host_grad", "muon_last_error",
+    "muon_step_batched_host_grad", "muon_last_error", "muon_selftest_wait_timeout",
 )
 
 
@@ -91,6 +91,7 @@ def _lib():
         "muon_timing_read": (c_int, [c_int, POINTER(c_double), POINTER(c_longlong), POINTER(c_double)]),
         "muon_status_string": (ctypes.c_char_p, [c_int]),
         "muon_last_error": (ctypes.c_char_p, []),
+        "muon_selftest_wait_timeout": (c_int, [c_void_p, c_size_t, c_void_p]),
         "muon_build_info": (ctypes.c_char_p, []),
         "muon_cayley_workspace_size": (c_size_t, [c_int, c_int, c_int]),
         "muon_cayley_step": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_float, c_float, c_int,

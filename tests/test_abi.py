@@ -196,3 +196,10 @@ def test_binding_rejects_tensors_it_cannot_pass_by_pointer():
         mb.ns_orthogonalize(torch.zeros((16, 8)).t(), torch.zeros((8, 16)), mb.Schedule.fixed(1), torch.zeros(1))
     with pytest.raises(ValueError, match="CUDA"):
         mb.stiefel_cayley_step(torch.zeros((16, 8)), torch.zeros((16, 8)), 0.01, torch.zeros(1))
+
+
+def test_wait_selftest_argument_errors_are_host_side():
+    lib = mb.load()
+    assert lib.muon_selftest_wait_timeout(None, 4096, None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_selftest_wait_timeout(ctypes.c_void_p(1 << 24), 100, None) == mb.MUON_ERR_INVALID_ARG
+    assert lib.muon_selftest_wait_timeout(ctypes.c_void_p((1 << 24) + 16), 4096, None) == mb.MUON_ERR_ALIGNMENT
