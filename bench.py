@@ -64,19 +64,59 @@ def cpu_cores():
     return os.cpu_count() or 1
 
 
-def oracle_sample(iters):
-    """fp64 oracle Muon step on one 4096x4096 matrix of the set (momentum, `iters` NS
-    iterations, update); returns (seconds, NS FLOP of the sample)."""
+LAYER_SHAPES = ((4096, 4096), (4096, 11008), (11008, 4096))   # distinct shapes of one Llama layer
+
+
+def layer_counts():
+    """How many matrices of each distinct shape one layer holds (4 attention projections,
+    2 up/gate, 1 down)."""
+    from matrix_orthogonalising_optimizer_02_b200 import workloads
+    layer = workloads.llama7b_shapes(1)
+    return {sh: layer.count(sh) for sh in LAYER_SHAPES}
+
+
+def oracle_shape_seconds(shape):
+    """Seconds of one fp64 oracle Muon step (momentum, 5 Newton-Schulz iterations, update)
+    on one matrix of `shape`, drawn like the set's (bf16 W ~ N(0, 0.02^2), G ~ N(0, 1e-3^2))."""
     import numpy as np
     import oracle as orc
     from matrix_orthogonalising_optimizer_02_b200 import workloads
     r = workloads.rng(1005)
-    W = orc.round_to_bf16(r.standard_normal((4096, 4096)) * 0.02)
-    G = orc.round_to_bf16(r.standard_normal((4096, 4096)) * 1e-3)
+    W = orc.round_to_bf16(r.standard_normal(shape) * 0.02)
+    G = orc.round_to_bf16(r.standard_normal(shape) * 1e-3)
     M = np.zeros_like(G)
     t0 = time.perf_counter()
-    orc.muon_step(W, G, M, lr=LR, beta=BETA, weight_decay=WD, schedule=orc.fixed_schedule(iters))
-    return time.perf_counter() - t0, ns_flops_algorithmic(4096, 4096, iters)
+    orc.muon_step(W, G, M, lr=LR, beta=BETA, weight_decay=WD, schedule=orc.fixed_schedule(5))
+    return time.perf_counter() - t0
+
+
+def oracle_set_ms(per_shape_s):
+    """The set's oracle time from per-shape step times: one layer is 4 x t(4096^2) +
+    2 x t(4096 x 11008) + t(11008 x 4096), and the set is LAYERS such layers (matrices are
+    stepped one after another, so their times add)."""
+    counts = layer_counts()
+    return 1e3 * LAYERS * sum(counts[sh] * per_shape_s[sh] for sh in LAYER_SHAPES)
+
+
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline_object(per_shape_s, kind="oracle"):
+    counts = layer_counts()
+    parts = ", ".join(f"{r}x{c}: {per_shape_s[(r, c)]:.2f} s" for (r, c) in LAYER_SHAPES)
+    return {"value": oracle_set_ms(per_shape_s), "unit": "ms", "cores": cpu_cores(), "kind": kind,
+            "cpu_model": cpu_model(),
+            "sample": "fp64 oracle full step (momentum, 5 NS iterations, update) timed on one matrix of each "
+                      f"distinct shape of a Llama-7B layer ({parts}); one layer = "
+                      + " + ".join(f"{counts[sh]} x t({sh[0]}x{sh[1]})" for sh in LAYER_SHAPES)
+                      + f", extrapolated x{LAYERS} layers"}
 
 
 def workload_config(shapes):
@@ -262,21 +302,25 @@ def _stiefel(gen):
     mb.stiefel_cayley_step(W, G, 1e-2, ws)
     torch.cuda.synchronize()
     mb.timing_enable(False)
-    kinds = {k: mb.timing_read(k) for k in ("tc_f32", "simt_gemm", "lu", "misc")}
-    work = kinds["tc_f32"][2] + kinds["simt_gemm"][2] + kinds["lu"][2]
+    kinds = {k: mb.timing_read(k) for k in ("tc_f32", "simt_gemm", "simt_gemm_f64", "lu", "misc")}
+    work = sum(kinds[k][2] for k in ("tc_f32", "simt_gemm", "simt_gemm_f64", "lu"))
     ms = _time_ms(lambda: mb.stiefel_cayley_step(W, G, 1e-2, ws), 1, 3)
-    # ALU roofline of the fp32 SIMT products: 148 SMs x 128 fp32 lanes x 2 FLOP per FMA at
-    # the maximum SM clock (1965 MHz) = 74.4 TFLOP/s
-    simt_ms, _, simt_work = kinds["simt_gemm"]
-    fp32_peak = 148 * 128 * 2 * 1.965e9 / 1e12
-    simt_tflops = simt_work / max(simt_ms * 1e-3, 1e-12) / 1e12
+    # ALU rooflines, one per arithmetic type, from the unit counts at the maximum SM clock
+    # (1965 MHz): 148 SMs x 128 fp32 FMA lanes x 2 FLOP = 74.4 TFLOP/s for the fp32 products,
+    # 148 SMs x 64 fp64 FMA lanes x 2 FLOP = 37.2 TFLOP/s for the fp64 LU and back-substitution
+    # updates
+    def roof(kind, lanes, what):
+        kms, _, kwork = kinds[kind]
+        peak = 148 * lanes * 2 * 1.965e9 / 1e12
+        ach = kwork / max(kms * 1e-3, 1e-12) / 1e12
+        return {"bound": "alu", "kernel": what, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "kernel_ms_per_step": kms,
+                "peak_source": f"148 SMs x {lanes} FMA lanes x 2 x 1965 MHz"}
     out["stiefel_16x4096x1024_step"] = {"ms": ms, "fma_tflops": work / (ms * 1e-3) / 1e12,
                                         "kernel_ms": {k: v[0] for k, v in kinds.items()},
                                         "tc_f32_tflops": kinds["tc_f32"][2] / max(kinds["tc_f32"][0] * 1e-3, 1e-12) / 1e12,
-                                        "roofline": {"bound": "alu", "kernel": "simt_gemm_kernel (fp32 and fp64 FMA)",
-                                                     "achieved": simt_tflops, "peak": fp32_peak, "unit": "TFLOP/s",
-                                                     "frac": simt_tflops / fp32_peak,
-                                                     "peak_source": "148 SMs x 128 fp32 FMA lanes x 2 x 1965 MHz"}}
+                                        "roofline_fp32": roof("simt_gemm", 128, "simt_gemm kernels, fp32 FMA products"),
+                                        "roofline_fp64": roof("simt_gemm_f64", 64, "simt_gemm_kernel<double>, fp64 FMA LU updates")}
     return out
 
 
@@ -290,29 +334,56 @@ def _single():
     hp1 = mb.hyper(lr=0.02, beta=0.95, weight_decay=0.0, schedule=mb.Schedule.fixed(5, fp32_mode=True))
     ws = mb.workspace(mb.muon_step_workspace_size(one, hp1))
     out["single_256x128_fp32_step_us"] = 1e3 * _time_ms(lambda: mb.muon_step_batched(one, hp1, ws), 5, 50)
+    # the device time of the step's kernels alone (events around each launch)
+    mb.timing_reset()
+    mb.timing_enable(True)
+    for _ in range(20):
+        mb.muon_step_batched(one, hp1, ws)
+    torch.cuda.synchronize()
+    mb.timing_enable(False)
+    kern_ms = sum(mb.timing_read(k)[0] for k in mb.KERNEL_KINDS)
+    launches = sum(mb.timing_read(k)[1] for k in mb.KERNEL_KINDS)
+    out["single_256x128_fp32_kernel_us"] = 1e3 * kern_ms / 20
+    out["single_256x128_fp32_launches"] = launches / 20
+    # the same step replayed from a CUDA graph (no host work per step)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        mb.muon_step_batched(one, hp1, ws, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        mb.muon_step_batched(one, hp1, ws)
+    out["single_256x128_fp32_graph_us"] = 1e3 * _time_ms(g.replay, 5, 50)
     return out
 
 
 def run_reference(args, rank, world):
-    """The oracle as it stands, on this host's cores: each step is one bounded sample (one
-    4096x4096 matrix: momentum, one NS iteration, update), extrapolated to the full set by
-    algorithmic NS FLOPs."""
+    """The oracle as it stands, on this host's cores.  Each step is one bounded sample: the
+    full oracle step on one matrix of one of the layer's three distinct shapes, the shapes
+    taken in turn.  The printed value is the set time composed from the mean time of each
+    shape over the timed steps (a shape that no timed step reached is timed once more after
+    them), exactly as the cpu_baseline of the device arm composes it."""
     if rank != 0:
         return
-    total = set_flops()
-    times = []
+    times = {sh: [] for sh in LAYER_SHAPES}
     for i in range(args.warmup + args.steps):
-        dt, fl = oracle_sample(1)
+        sh = LAYER_SHAPES[i % len(LAYER_SHAPES)]
+        dt = oracle_shape_seconds(sh)
         if i >= args.warmup:
-            times.append(dt * total / fl)
-    ms = 1e3 * statistics.mean(times)
-    sample = "one 4096x4096 matrix of the set per step (momentum, 1 of 5 NS iterations, update), " \
-             "extrapolated to the 224-matrix set by algorithmic NS FLOP"
+            times[sh].append(dt)
+    for sh in LAYER_SHAPES:
+        if not times[sh]:
+            times[sh].append(oracle_shape_seconds(sh))
+    per_shape = {sh: statistics.mean(v) for sh, v in times.items()}
+    ms = oracle_set_ms(per_shape)
+    base = cpu_baseline_object(per_shape)
+    base["sample"] += f"; {args.steps} timed steps take the three shapes in turn"
     out = {"metric": "Muon full-step ms per param set (Llama-7B-shaped set)", "value": ms, "unit": "ms",
            "impl": "reference", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic", "config": workload_config(set_shapes()),
-           "cpu_baseline": {"value": ms, "unit": "ms", "cores": cpu_cores(), "kind": "oracle", "sample": sample},
+           "cpu_baseline": base,
            "e2e": {"value": ms, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -484,11 +555,7 @@ def main():
         torch.cuda.empty_cache()
         out["secondary"] = secondary_measurements()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, fl = oracle_sample(5)
-        out["cpu_baseline"] = {"value": 1e3 * dt * total_flops / fl, "unit": "ms", "cores": cpu_cores(),
-                               "kind": "oracle",
-                               "sample": "one 4096x4096 matrix, full step (momentum, 5 NS iterations, update) "
-                                         f"in {dt:.1f} s, extrapolated to the set by algorithmic NS FLOP"}
+        out["cpu_baseline"] = cpu_baseline_object({sh: oracle_shape_seconds(sh) for sh in LAYER_SHAPES})
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -65,7 +65,14 @@ typedef enum {
     MUON_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the *_workspace_size() minimum    */
     MUON_ERR_CUDA = 5,                 /* a CUDA runtime/driver call failed               */
     MUON_ERR_NONFINITE = 6,            /* device status: a NaN/Inf Frobenius norm          */
-    MUON_ERR_DEVICE_TIMEOUT = 7        /* device status: a kernel wait gave up (bounded)  */
+    MUON_ERR_DEVICE_TIMEOUT = 7,       /* device status: a kernel wait gave up (bounded); the
+                                          kernel drained its copies and MMAs in flight before
+                                          it released its memory, so the context stays usable */
+    MUON_ERR_DEVICE_UNDRAINED = 8      /* device status: a wait gave up AND copies or MMAs
+                                          already in flight did not finish within the drain
+                                          limit (100 ms) before the kernel released its shared
+                                          and tensor memory.  Results are undefined and the
+                                          CUDA context should not be trusted: end the process */
 } muon_status;
 
 typedef enum { MUON_BF16 = 0, MUON_F32 = 1 } muon_dtype;
@@ -187,7 +194,12 @@ MUON_API muon_status stiefel_cayley_step(float* W, const float* G, int batch, in
  * at zero (each slot is written before it is read within a call).  Calls that overlap on
  * the GPU (e.g. on two streams) race on the array and must be ordered by the caller.
  * Limits: batch <= MUON_STATIC_MAX_BATCH and batch * ceil(rows*cols / 8192) <=
- * MUON_STATIC_MAX_BLOCKS, else MUON_ERR_UNSUPPORTED_SHAPE.  Pointers need no alignment. */
+ * MUON_STATIC_MAX_BLOCKS, else MUON_ERR_UNSUPPORTED_SHAPE.  Pointers need no alignment.
+ * X_out may equal X_in when in_dtype == out_dtype (each element is read before it is
+ * written, by the same thread); other overlaps are not allowed.
+ * A non-finite input is not reported (there is no status word): a matrix with an infinite
+ * element gets scale 0 and NaN at that element, one with a NaN gets a NaN scale and NaN
+ * everywhere.  Callers that need the check pass scale_out and test it for 0 or NaN. */
 #define MUON_STATIC_MAX_BLOCKS 65536
 #define MUON_STATIC_MAX_BATCH 4096
 MUON_API muon_status muon_frobenius_prescale_static(const void* X_in, int in_dtype, void* X_out, int out_dtype,
@@ -215,7 +227,9 @@ MUON_API muon_status muon_cayley_step(float* W, const float* G, float* M, int ba
                                       float beta, int center, void* workspace, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then reads the device-side status word of `workspace` into
- * *status_out (MUON_OK, MUON_ERR_NONFINITE or MUON_ERR_DEVICE_TIMEOUT) and clears it. */
+ * *status_out and clears it: MUON_ERR_DEVICE_UNDRAINED if any kernel gave up a wait and
+ * could not drain, else MUON_ERR_DEVICE_TIMEOUT if a wait gave up, else MUON_ERR_NONFINITE
+ * if a norm or pivot was not finite, else MUON_OK. */
 MUON_API muon_status muon_workspace_device_status(void* workspace, size_t ws_bytes, int* status_out,
                                          void* stream);
 
@@ -233,7 +247,9 @@ typedef enum {
     MUON_KERNEL_LU = 5,           /* 2k x 2k LU and triangular solves                     */
     MUON_KERNEL_MISC = 6,         /* casts, copies, block assembly, plane splits          */
     MUON_KERNEL_TC_F32 = 7,       /* tcgen05 fp32 products from three bf16 planes (Stiefel) */
-    MUON_KERNEL_KINDS = 8
+    MUON_KERNEL_SIMT_GEMM_F64 = 8,  /* fp64 DFMA GEMMs (Stiefel LU trailing updates and
+                                       back substitution)                                  */
+    MUON_KERNEL_KINDS = 9
 } muon_kernel_kind;
 MUON_API muon_status muon_timing_enable(int enable);
 MUON_API muon_status muon_timing_reset(void);

@@ -19,11 +19,12 @@ LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
 # enums of muon_b200.h
 MUON_OK, MUON_ERR_INVALID_ARG, MUON_ERR_UNSUPPORTED_SHAPE, MUON_ERR_ALIGNMENT = 0, 1, 2, 3
 MUON_ERR_WORKSPACE_TOO_SMALL, MUON_ERR_CUDA, MUON_ERR_NONFINITE, MUON_ERR_DEVICE_TIMEOUT = 4, 5, 6, 7
+MUON_ERR_DEVICE_UNDRAINED = 8
 MUON_BF16, MUON_F32 = 0, 1
 SCALE_MODES = {"moonlight": 0, "kellerjordan": 1, "mup": 2, "naive": 3}
 MUON_MAX_NS_ITERS = 32
 KERNEL_KINDS = {"momentum": 0, "scale": 1, "ns_gemm": 2, "update": 3, "simt_gemm": 4, "lu": 5, "misc": 6,
-                "tc_f32": 7}
+                "tc_f32": 7, "simt_gemm_f64": 8}
 
 #: Exported entry points, as declared in include/muon_b200.h.
 EXPORTED = (

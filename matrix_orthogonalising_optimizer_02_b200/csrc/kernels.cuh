@@ -11,6 +11,9 @@ namespace muon {
 // Device status bits (first word of every workspace).
 constexpr unsigned kDevErrTimeout = 1u;
 constexpr unsigned kDevErrNonfinite = 2u;
+// After a timeout, copies or MMAs already issued did not finish within the drain limit
+// before the kernel released its shared and tensor memory.
+constexpr unsigned kDevErrUndrained = 4u;
 
 // ------------------------------------------------------------------ tcgen05 grouped GEMM
 // One problem of a grouped launch: out = f * (alpha * (A_op x B_op) + beta * E), f = 1 or
@@ -137,6 +140,33 @@ struct alignas(16) UpdateItem {
     int vec;
 };
 cudaError_t update_launch(const UpdateItem* d_items, int count, long long total_blocks, cudaStream_t stream);
+
+// ------------------------------------------------------------------ fused small fp32 step
+// One cluster of kSmallCluster CTAs per matrix runs momentum, Frobenius pre-scale, every
+// Newton-Schulz iteration and the update of an fp32-mode matrix with r = min(rows, cols) <=
+// kSmallMaxR (r % 8 == 0) and ceil(max(rows, cols) / kSmallCluster) <= kSmallMaxR.
+constexpr int kSmallCluster = 8, kSmallThreads = 256, kSmallMaxR = 128;
+struct alignas(16) SmallItem {
+    const void* G;   // gradient (step) or input X (orthogonalisation only); bf16 or fp32
+    float* M;        // momentum, updated in place; nullptr: X0 = G
+    void* W;         // weights, updated in place; nullptr: no update
+    void* O;         // optional copy of the orthogonalised matrix
+    int rows, cols;
+    int g_f32, w_f32, o_f32;
+    float decay;     // 1 - lr*wd
+    float step;      // -lr*scale
+};
+struct SmallParams {
+    float beta;
+    int nesterov;
+    float eps;
+    int n_iters;
+    float coeffs[3 * 32];
+};
+bool ns_small_fits(int rows, int cols);
+size_t ns_small_smem_bytes();
+cudaError_t ns_small_launch(const SmallItem* d_items, int count, const SmallParams& prm, unsigned* d_status,
+                            cudaStream_t stream);
 
 // dst (dtype dst_f32) = f * src (bf16 or fp32), f = *dscale or 1; batched items.
 struct alignas(16) CastItem {

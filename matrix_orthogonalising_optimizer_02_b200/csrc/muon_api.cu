@@ -316,6 +316,17 @@ muon_status build_ns_simt(Plan& plan, TableImage& img, std::vector<NsMat>& mats,
     return MUON_OK;
 }
 
+SmallParams small_params(const muon_ns_schedule& sch, float beta, int nesterov) {
+    SmallParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.beta = beta;
+    prm.nesterov = nesterov;
+    prm.eps = sch.eps;
+    prm.n_iters = sch.n_iters;
+    for (int i = 0; i < 3 * sch.n_iters; ++i) prm.coeffs[i] = sch.coeffs[i];
+    return prm;
+}
+
 float scale_for(int rows, int cols, int mode) {
     const double d_out = rows, d_in = cols;
     switch (mode) {
@@ -497,6 +508,7 @@ const char* muon_status_string(muon_status s) {
         case MUON_ERR_CUDA: return "CUDA error";
         case MUON_ERR_NONFINITE: return "non-finite Frobenius norm";
         case MUON_ERR_DEVICE_TIMEOUT: return "a device wait timed out";
+        case MUON_ERR_DEVICE_UNDRAINED: return "a device wait timed out and work in flight did not drain";
     }
     return "unknown status";
 }
@@ -552,10 +564,38 @@ muon_status step_batched(const muon_matrix_desc* descs, int count, const muon_hy
     unsigned* d_status = static_cast<unsigned*>(workspace);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
 
+    // fp32 mode on small matrices: the whole step of each matrix in one cluster (one launch)
+    bool small = H.ns.fp32_mode != 0;
+    for (int i = 0; i < count && small; ++i) small = ns_small_fits(D[i].rows, D[i].cols);
+
     auto build = [&](Plan& plan, TableImage& img) -> muon_status {
         muon_ns_schedule sch = H.ns;
         sch.coeffs = coeffs.data();
         const bool fp32 = sch.fp32_mode != 0;
+        if (small) {
+            std::vector<SmallItem> items;
+            double flops = 0.0;
+            for (int i = 0; i < count; ++i) {
+                const muon_matrix_desc& d = D[i];
+                SmallItem it;
+                std::memset(&it, 0, sizeof(it));
+                it.G = d.G; it.M = d.M; it.W = d.W; it.O = d.O_out;
+                it.rows = d.rows; it.cols = d.cols;
+                it.g_f32 = d.g_dtype == MUON_F32; it.w_f32 = d.w_dtype == MUON_F32; it.o_f32 = 1;
+                it.decay = 1.0f - H.lr * H.weight_decay;
+                it.step = -H.lr * scale_for(d.rows, d.cols, H.scale_mode);
+                items.push_back(it);
+                const double r = std::min(d.rows, d.cols), sdim = std::max(d.rows, d.cols);
+                flops += sch.n_iters * (3.0 * r * r * sdim + r * r * r);
+            }
+            const SmallItem* di = img.dev<SmallItem>(img.add(items.data(), items.size() * sizeof(SmallItem), kAlign));
+            const SmallParams prm = small_params(sch, H.beta, H.nesterov);
+            plan.steps.push_back({MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t st) {
+                                      return ns_small_launch(di, count, prm, d_status, st);
+                                  }});
+            if (img.bytes.size() > L.table_bound) return MUON_ERR_WORKSPACE_TOO_SMALL;
+            return MUON_OK;
+        }
         for (const auto& g : L.groups) {
             Arena ar;
             ar.base = ws + kHeaderBytes;
@@ -760,9 +800,32 @@ muon_status ns_orthogonalize(const void* X_in, int in_dtype, void* X_out, int ou
     unsigned* d_status = static_cast<unsigned*>(workspace);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
 
+    const bool small = fp32 && ns_small_fits(rows, cols);
     auto build = [&](Plan& plan, TableImage& img) -> muon_status {
         muon_ns_schedule sch = S;
         sch.coeffs = coeffs.data();
+        if (small) {   // fp32 mode on small matrices: one cluster per matrix, one launch
+            std::vector<SmallItem> items;
+            const size_t in_es = in_dtype == MUON_F32 ? 4 : 2, out_es = out_dtype == MUON_F32 ? 4 : 2;
+            for (int i = 0; i < batch; ++i) {
+                SmallItem it;
+                std::memset(&it, 0, sizeof(it));
+                it.G = static_cast<const uint8_t*>(X_in) + static_cast<size_t>(i) * n * in_es;
+                it.O = static_cast<uint8_t*>(X_out) + static_cast<size_t>(i) * n * out_es;
+                it.rows = rows; it.cols = cols;
+                it.g_f32 = in_dtype == MUON_F32; it.o_f32 = out_dtype == MUON_F32;
+                items.push_back(it);
+            }
+            const SmallItem* di = img.dev<SmallItem>(img.add(items.data(), items.size() * sizeof(SmallItem), kAlign));
+            const SmallParams prm = small_params(sch, 0.f, 0);
+            const double r = std::min(rows, cols), sdim = std::max(rows, cols);
+            const double flops = static_cast<double>(batch) * sch.n_iters * (3.0 * r * r * sdim + r * r * r);
+            plan.steps.push_back({MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t st) {
+                                      return ns_small_launch(di, batch, prm, d_status, st);
+                                  }});
+            if (table_offset + img.bytes.size() > ws_bytes) return MUON_ERR_WORKSPACE_TOO_SMALL;
+            return MUON_OK;
+        }
         Arena ar;
         ar.base = ws + kHeaderBytes;
         double* partials = static_cast<double*>(ar.at(ar.take(static_cast<size_t>(nb1 * batch) * sizeof(double))));
@@ -840,7 +903,10 @@ muon_status muon_workspace_device_status(void* workspace, size_t ws_bytes, int* 
     if (cudaStreamSynchronize(stream) != cudaSuccess) return MUON_ERR_CUDA;
     if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MUON_ERR_CUDA;
     if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MUON_ERR_CUDA;
-    *status_out = (word & kDevErrTimeout) ? MUON_ERR_DEVICE_TIMEOUT : (word & kDevErrNonfinite) ? MUON_ERR_NONFINITE : MUON_OK;
+    *status_out = (word & kDevErrUndrained)   ? MUON_ERR_DEVICE_UNDRAINED
+                  : (word & kDevErrTimeout)   ? MUON_ERR_DEVICE_TIMEOUT
+                  : (word & kDevErrNonfinite) ? MUON_ERR_NONFINITE
+                                              : MUON_OK;
     return MUON_OK;
 }
 

@@ -149,7 +149,8 @@ muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t
         if (st != MUON_OK) return st;
     }
     static const char* const kind_names[MUON_KERNEL_KINDS] = {"momentum", "scale", "ns_gemm", "update",
-                                                              "simt_gemm", "lu", "misc", "tc_f32"};
+                                                              "simt_gemm", "lu", "misc", "tc_f32",
+                                                              "simt_gemm_f64"};
     for (size_t si = 0; si < plan->steps.size(); ++si) {
         const PlanStep& s = plan->steps[si];
         if (g_timing.enabled) {

@@ -35,8 +35,9 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     lib = mb.load()
-    for s in range(8):
-        assert lib.muon_status_string(s)
+    for s in range(9):
+        assert lib.muon_status_string(s) != b"unknown status"
+    assert lib.muon_status_string(9) == b"unknown status"
     assert b"sm_100a" in lib.muon_build_info()
 
 

@@ -14,7 +14,7 @@ import torch
 import oracle as orc
 from matrix_orthogonalising_optimizer_02_b200 import binding as mb
 from matrix_orthogonalising_optimizer_02_b200 import workloads
-from gpu_helpers import bf16_ulp_diff, dev, host, rel_f, sv
+from gpu_helpers import assert_update_within_bound, dev, host, rel_f, sv, sv_gram
 
 pytestmark = pytest.mark.gpu
 
@@ -49,11 +49,10 @@ def _check_set(shapes, seed, sample):
         O = host(m.O_out)
         O_ref = orc.newton_schulz(orc.ns_input(M1), orc.fixed_schedule(5))
         assert rel_f(O, O_ref) <= 2e-2
-        if O.shape[0] == O.shape[1] or max(O.shape) <= 3072:
-            assert np.max(np.abs(sv(O) - sv(O_ref))) <= 0.05
+        # the bf16 bound on every sampled shape, the 4096 x 11008 and 11008 x 4096 included
+        assert np.max(np.abs(sv_gram(O) - sv_gram(O_ref))) <= 0.05
         s = orc.scale_factor(*W0.shape, "moonlight")
-        R = orc.round_to_bf16(orc.muon_update(W0, O, LR, WD, s))
-        assert np.mean(bf16_ulp_diff(host(m.W), R) <= 1) > 0.999
+        assert_update_within_bound(host(m.W), W0, O, LR, WD, s, bf16=True)
     # every matrix of the set: finite weights and momentum after the step
     for m in mats:
         assert torch.isfinite(m.W.float()).all() and torch.isfinite(m.M).all()

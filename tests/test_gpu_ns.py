@@ -80,6 +80,32 @@ def test_ns_fp32_mode(shape):
     assert rel_f(got, want) <= FP32_TOL
 
 
+@pytest.mark.parametrize("shape", [(128, 1024), (1024, 128), (96, 40), (40, 96), (8, 16), (120, 120)])
+def test_ns_fp32_small_fused(shape):
+    """fp32 mode with min(rows, cols) <= 128 runs as one cluster per matrix: the largest long
+    side (1024 = 8 slabs of 128), tall and wide, slabs of 5 columns, a tiny matrix and a
+    square one, batched, each against the oracle."""
+    r = workloads.rng(410 + shape[0] + 3 * shape[1])
+    X = dev(r.standard_normal((3, *shape)) * 0.02, torch.float32)
+    got = run_ns(X, mb.Schedule.fixed(5, fp32_mode=True), out_dtype=torch.float32)
+    for i in range(3):
+        want = orc.newton_schulz(host(X[i]), orc.fixed_schedule(5))
+        assert rel_f(host(got[i]), want) <= FP32_TOL
+    one = run_ns(X[1].contiguous(), mb.Schedule.fixed(5, fp32_mode=True), out_dtype=torch.float32)
+    assert torch.equal(one, got[1])
+
+
+def test_ns_fp32_small_fused_bf16_io_and_hybrid():
+    """bf16 input and output around the fp32 iteration, under the 10-iteration hybrid
+    schedule."""
+    r = workloads.rng(420)
+    X = dev(r.standard_normal((2, 64, 200)), torch.bfloat16)
+    got = run_ns(X, mb.Schedule.hybrid(fp32_mode=True), out_dtype=torch.bfloat16)
+    for i in range(2):
+        want = orc.newton_schulz(host(X[i]), orc.hybrid_schedule())
+        assert rel_f(host(got[i]), want) <= 4e-3       # one bf16 rounding of the output
+
+
 @pytest.mark.parametrize("sched,nsplit", [("kj5", 2), ("hybrid", 4)])
 def test_ns_low_rank_split(sched, nsplit):
     G = workloads.low_rank_plus_noise(batch=2, n=1024)

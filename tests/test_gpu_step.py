@@ -12,7 +12,7 @@ import torch
 import oracle as orc
 from matrix_orthogonalising_optimizer_02_b200 import binding as mb
 from matrix_orthogonalising_optimizer_02_b200 import workloads
-from gpu_helpers import bf16_ulp_diff, dev, f32_ulp_diff, host, rel_f
+from gpu_helpers import assert_update_within_bound, dev, f32_ulp_diff, host, rel_f
 
 pytestmark = pytest.mark.gpu
 
@@ -49,18 +49,7 @@ def check_step(mats, before, lr, wd, beta, nesterov, scale_mode, sched_host, fp3
         O_ref = orc.newton_schulz(X0, sched_host) if sched_host else orc.frobenius_prescale(X0)
         assert rel_f(O, O_ref) <= (1e-4 if fp32 else 2e-2)
         s = orc.scale_factor(rows, cols, scale_mode)
-        W1_ref = orc.muon_update(W0, O, lr, wd, s)
-        W1 = host(m.W)
-        # fp32 evaluation of decay*W0 + step*O rounds twice (|err| <= 2^-23 per term), then
-        # the weight is stored: within one storage ulp of the exact value plus that error.
-        f32_err = 2.0 ** -23 * (np.abs((1 - lr * wd) * W0) + np.abs(lr * s * O))
-        if m.W.dtype == torch.bfloat16:
-            R = orc.round_to_bf16(W1_ref)
-            ulp = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(R), 1e-38))) - 7), 2.0 ** -133)
-            assert np.all(np.abs(W1 - R) <= ulp + f32_err)
-            assert np.mean(bf16_ulp_diff(W1, R) == 0) > 0.99
-        else:
-            assert np.all(np.abs(W1 - W1_ref) <= 2.0 ** -23 * np.abs(W1_ref) + f32_err)
+        assert_update_within_bound(host(m.W), W0, O, lr, wd, s, m.W.dtype == torch.bfloat16)
 
 
 def test_step_single_fp32_matrix():
@@ -76,6 +65,29 @@ def test_step_single_fp32_matrix():
     # and the whole oracle step
     ref = orc.muon_step(W, G, M, lr=0.02, beta=0.95, fp32_mode=True, w_dtype="f32")
     assert rel_f(host(mats[0].O_out), ref["O"]) <= 1e-4
+
+
+@pytest.mark.parametrize("nesterov", [False, True])
+def test_step_fp32_small_fused_mixed_set(nesterov):
+    """fp32 mode on a mixed set of small matrices (one fused launch): bf16 and fp32 weights
+    and gradients, non-zero momentum, weight decay, tall, wide and ragged slabs."""
+    shapes = [(256, 128), (128, 256), (64, 200), (200, 64), (8, 16)]
+    mats = []
+    r = workloads.rng(17)
+    for i, (rows, cols) in enumerate(shapes):
+        wd = torch.bfloat16 if i % 2 else torch.float32
+        gd = torch.float32 if i % 3 else torch.bfloat16
+        mats.append(mb.Matrix(dev(r.standard_normal((rows, cols)) * 0.02, wd),
+                              dev(r.standard_normal((rows, cols)) * 1e-3, gd),
+                              dev(r.standard_normal((rows, cols)) * 1e-3, torch.float32),
+                              torch.empty((rows, cols), dtype=torch.float32, device="cuda")))
+    hp = mb.hyper(lr=0.02, beta=0.95, weight_decay=0.1, nesterov=nesterov,
+                  schedule=mb.Schedule.fixed(5, fp32_mode=True))
+    before = snapshot(mats)
+    ws = mb.workspace(mb.muon_step_workspace_size(mats, hp))
+    mb.muon_step_batched(mats, hp, ws)
+    assert mb.device_status(ws) == mb.MUON_OK
+    check_step(mats, before, 0.02, 0.1, 0.95, nesterov, "moonlight", orc.fixed_schedule(5), fp32=True)
 
 
 @pytest.mark.parametrize("nesterov", [False, True])

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as orc
 from matrix_orthogonalising_optimizer_02_b200 import binding as mb
 from matrix_orthogonalising_optimizer_02_b200 import workloads
 
@@ -33,6 +34,17 @@ def _reference(X, out_dtype, fp32_mode):
     mb.ns_orthogonalize(X, Y, sch, ws)
     assert mb.device_status(ws) == mb.MUON_OK
     return Y
+
+
+def _dt(t):
+    return mb.MUON_F32 if t == torch.float32 else mb.MUON_BF16
+
+
+def _call(lib, x_ptr, din, y_ptr, dout, batch, rows, cols, fp32, scale=None):
+    return lib.muon_frobenius_prescale_static(
+        x_ptr, _dt(din), y_ptr, _dt(dout), batch, rows, cols, int(fp32), ctypes.c_float(1e-7),
+        ctypes.c_void_p(scale.data_ptr() if scale is not None else None),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
 def test_static_prescale_two_calls_match_workspace_path():
@@ -66,3 +78,63 @@ def test_static_prescale_rejects_sizes_beyond_the_scratch():
     st = lib.muon_frobenius_prescale_static(X.data_ptr(), mb.MUON_F32, X.data_ptr(), mb.MUON_F32, 5000, 8, 8,
                                             0, ctypes.c_float(1e-7), None, None)
     assert st == mb.MUON_ERR_UNSUPPORTED_SHAPE
+
+
+def test_static_prescale_matches_the_oracle():
+    """One bf16 case against the oracle's Frobenius pre-scale of the rounded input."""
+    lib = mb.load()
+    r = workloads.rng(710)
+    X = torch.tensor(r.standard_normal((2, 96, 160)), dtype=torch.float32).to(torch.bfloat16).cuda()
+    Y = torch.empty(X.shape, dtype=torch.float32, device="cuda")
+    assert _call(lib, X.data_ptr(), torch.bfloat16, Y.data_ptr(), torch.float32, 2, 96, 160, False) == mb.MUON_OK
+    torch.cuda.synchronize()
+    for i in range(2):
+        want = orc.frobenius_prescale(X[i].double().cpu().numpy())
+        got = Y[i].double().cpu().numpy()
+        # fp32 partial sums of 32 squares per thread (relative error below 2^-19 in the squared
+        # norm), one rounding of the fp32 scale and one of the product
+        assert np.max(np.abs(got - want)) <= 1e-5 * np.max(np.abs(want))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_static_prescale_unaligned_and_in_place(dtype):
+    """Pointers one element past an aligned base, and X_out == X_in, against the workspace
+    path on an aligned copy of the same values."""
+    lib = mb.load()
+    batch, rows, cols = 2, 72, 136
+    r = workloads.rng(711)
+    n = batch * rows * cols
+    base_in = torch.tensor(r.standard_normal(n + 1), dtype=torch.float32).to(dtype).cuda()
+    X = base_in[1:].view(batch, rows, cols)                     # one element off the allocation
+    ref = _reference(X.contiguous().clone(), dtype, False)
+    base_out = torch.full((n + 1,), float("nan"), dtype=dtype, device="cuda")
+    Y = base_out[1:].view(batch, rows, cols)
+    assert _call(lib, X.data_ptr(), dtype, Y.data_ptr(), dtype, batch, rows, cols, False) == mb.MUON_OK
+    torch.cuda.synchronize()
+    assert torch.allclose(Y.double(), ref.double(), rtol=1e-6, atol=0.0)
+    Z = X.clone()
+    assert _call(lib, Z.data_ptr(), dtype, Z.data_ptr(), dtype, batch, rows, cols, False) == mb.MUON_OK
+    torch.cuda.synchronize()
+    assert torch.allclose(Z.double(), ref.double(), rtol=1e-6, atol=0.0)
+
+
+def test_static_prescale_nonfinite_input_shows_in_the_scale():
+    """No status word: an infinite element gives scale 0 (and NaN at that element), a NaN
+    gives a NaN scale; the other matrix of the batch is unaffected."""
+    lib = mb.load()
+    r = workloads.rng(712)
+    for bad, want_scale in ((float("inf"), 0.0), (float("nan"), None)):
+        X = torch.tensor(r.standard_normal((2, 64, 64)), dtype=torch.float32).cuda()
+        X[0, 3, 5] = bad
+        Y = torch.empty_like(X)
+        scale = torch.full((2,), 7.0, dtype=torch.float32, device="cuda")
+        assert _call(lib, X.data_ptr(), torch.float32, Y.data_ptr(), torch.float32, 2, 64, 64, False,
+                     scale) == mb.MUON_OK
+        torch.cuda.synchronize()
+        s0 = float(scale[0])
+        if want_scale is None:
+            assert np.isnan(s0) and torch.isnan(Y[0]).all()
+        else:
+            assert s0 == want_scale and torch.isnan(Y[0, 3, 5]) and int(torch.isnan(Y[0]).sum()) == 1
+        x1 = X[1].to(torch.bfloat16).double()
+        assert abs(float(scale[1]) - 1.0 / (float(x1.norm()) + 1e-7)) <= 1e-6 * float(scale[1])
