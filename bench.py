@@ -127,25 +127,21 @@ def workload_config(shapes):
 
 
 def recorded_traffic(layers_per_launch):
-    """DRAM bytes per NS GEMM launch: the committed ncu summary's per-launch bytes on one
-    layer (7 independent matrices, so traffic grows in proportion) times the layers one launch
-    covers, if the summary was captured on the kernel sources as they are now (else None)."""
+    """DRAM bytes per NS GEMM launch: the per-launch bytes ncu recorded on one layer (7
+    independent matrices, so traffic grows in proportion), from profiles/tc_gemm_traffic.json,
+    times the layers one launch covers -- if that capture was made on the kernel sources as
+    they are now (else None)."""
     import hashlib
-    md = os.path.join(ROOT, "profiles", "tc_gemm_llama7b_1layer.md")
-    if not os.path.exists(md):
+    path = os.path.join(ROOT, "profiles", "tc_gemm_traffic.json")
+    if not os.path.exists(path):
         return None
-    fields = {}
-    for line in open(md):
-        if ":" in line and line.split(":")[0].strip() in ("traffic_bytes_per_launch_one_layer",
-                                                           "kernel_source_sha256_16"):
-            k, v = line.split(":", 1)
-            fields[k.strip()] = v.strip()
+    rec = json.load(open(path))
     h = hashlib.sha256()
-    for f in ("tc_gemm.cu", "kernels.cuh", "ptx_sm100.cuh"):
-        h.update(open(os.path.join(ROOT, "matrix_orthogonalising_optimizer_02_b200", "csrc", f), "rb").read())
-    if fields.get("kernel_source_sha256_16") != h.hexdigest()[:16] or "traffic_bytes_per_launch_one_layer" not in fields:
+    for f in rec.get("kernel_sources", []):
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if rec.get("kernel_source_sha256_16") != h.hexdigest()[:16] or "traffic_bytes_per_launch_one_layer" not in rec:
         return None
-    return int(int(fields["traffic_bytes_per_launch_one_layer"]) * layers_per_launch)
+    return int(rec["traffic_bytes_per_launch_one_layer"] * layers_per_launch)
 
 
 def set_flops():

@@ -36,7 +36,11 @@ constexpr int MN_CHUNK_BYTES = 64 * BK * 2;          // one 64(MN) x 64(K) box: 
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COLS = 256;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+// Per epilogue warp, 32 x 32 bf16 chunks (64-byte rows): one for the direct store, one for the
+// transposed mirror, and two for E (the chunk in use and the one being fetched).
+constexpr int STG_BYTES = 32 * 64;
+constexpr int STG_WARP_BYTES = 4 * STG_BYTES;
+constexpr int SMEM_TOTAL = STAGES * STAGE_BYTES + BAR_BYTES + (kTcEpilogueThreads / 32) * STG_WARP_BYTES + 1024;
 static_assert(SMEM_TOTAL <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 static_assert(HM == 128 && HN == 128, "pair tile is 256 x 256");
 
@@ -56,6 +60,24 @@ __device__ __forceinline__ void segment_planes(const TcProblem& P, int seg, int&
     pa = static_cast<int>(c & 3u);
     pb = static_cast<int>(c >> 2);
 }
+
+// Byte offset of 16-byte segment `seg` (0..3) of row `row` in a 32 x 64-byte staging chunk,
+// segments XOR-swizzled by (row >> 1) & 3: a warp touching one segment of 32 rows, or 4
+// segments of 8 rows, hits every bank group once per 8 lanes (no conflicts).
+__device__ __forceinline__ int stg_off64(int row, int seg) { return row * 64 + 16 * (seg ^ ((row >> 1) & 3)); }
+
+// 16-byte global -> shared copy (cp.async, L2 only); bytes past src_bytes are zero-filled.
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gmem_src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
     uint4 w;
@@ -170,9 +192,11 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             for (int s = 0; s < STAGES; ++s) {
                 if (issued_parity[s] < 0) continue;
                 const unsigned long long t0 = global_ns();
-                while (!mbar_try_wait(&full_bar[s], static_cast<uint32_t>(issued_parity[s])) &&
+                bool landed = false;
+                while (!(landed = mbar_try_wait(&full_bar[s], static_cast<uint32_t>(issued_parity[s]))) &&
                        global_ns() - t0 < 100000000ull) {
                 }
+                if (!landed) atomicOr(dev_status, kDevErrUndrained);
             }
         }
     } else if (warp == 1 && lane == 0 && rank == 0) {
@@ -217,17 +241,30 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             // Drain: wait (bounded) until every MMA issued so far has finished.
             tc_commit_pair(&tfull_bar[acc], 0x3);
             const unsigned long long t0 = global_ns();
-            while (!mbar_try_wait(&tfull_bar[acc], acc_phase) && global_ns() - t0 < 100000000ull) {
+            bool done = false;
+            while (!(done = mbar_try_wait(&tfull_bar[acc], acc_phase)) && global_ns() - t0 < 100000000ull) {
             }
+            if (!done) atomicOr(dev_status, kDevErrUndrained);
         }
     } else if (warp >= 4) {
         // ------------------------------------------------------------ epilogue
         // 8 warps: warp & 3 selects the TMEM lane quarter (rows), (warp - 4) >> 2 the half of
-        // the 256 columns.  E (the a*X / b*A / fp32 addend) is prefetched one 32-column
-        // chunk ahead as raw 16-byte words, the first chunk before the accumulator wait.
+        // the 256 columns.  tcgen05.ld gives lane L row L of a 32 x 32 chunk.  For bf16 E and
+        // outputs every global access is coalesced: E is fetched as 8 rows x 64 B per
+        // instruction and turned into rows through this warp's staging buffer, results go back
+        // through it and out as 8 rows x 64 B per instruction, and the mirror of a symmetric
+        // output is transposed there.  (A lane-per-row access touches 32 lines per instruction;
+        // measured on the Llama-7B set, that traffic alone lowered the power-capped clock from
+        // 1.94 to 1.46 GHz.)  fp32 problems and chunks on the diagonal of a symmetric output
+        // keep per-lane accesses (the diagonal needs per-element masks).  E is prefetched one
+        // chunk ahead, the first chunk before the accumulator wait.
         const int q = warp & 3;
         const int c_beg = ((warp - 4) >> 2) * (BN / 64);
         const int c_end = c_beg + BN / 64;
+        uint8_t* stg = smem + STAGES * STAGE_BYTES + BAR_BYTES + (warp - 4) * STG_WARP_BYTES;   // direct stores
+        uint8_t* stg_t = stg + STG_BYTES;              // transposed chunk of a mirror store
+        uint8_t* stg_e = stg + 2 * STG_BYTES;          // E of two chunks (double buffer)
+        const int crow = lane >> 2, cseg = lane & 3;   // coalesced layout: rows crow + 8i, segment cseg
         uint32_t acc = 0, acc_phase = 0;
         for (int t = pair; t < num_tiles; t += npairs) {
             const TileInfo ti = decode(tiles[t]);
@@ -242,144 +279,291 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
             const bool sym = (P.flags & kProbSym) != 0;
             const bool out_f32 = (P.flags & kProbOutF32) != 0;
             const bool e_f32 = (P.flags & kProbEF32) != 0;
-            const int row = ti.m0 + HM * static_cast<int>(rank) + q * 32 + lane;
+            const int row0 = ti.m0 + HM * static_cast<int>(rank) + q * 32;
+            const int row = row0 + lane;
             const bool row_ok = row < P.M;
             const bool has_e = (beta != 0.0f) && (P.E[0] != nullptr);
             const bool e_lo = has_e && !e_f32 && (P.E[1] != nullptr);
             const bool lo_out = !out_f32 && P.out[1] != nullptr;
             const size_t row_base = static_cast<size_t>(row) * P.ld;
-            // E of chunk c for this row: bf16 -> ew[0..3] plane 0, ew[4..7] plane 1; fp32 -> ew[0..7]
-            auto load_e = [&](int c, uint4 (&ew)[8]) {
-                const int col0 = ti.n0 + c * 32;
-                const bool need = has_e && row_ok && col0 < P.N && (!sym || col0 + 31 >= row);
+            const uint32_t t_row = tmem_base + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
+
+            // v[32] = alpha * acc + beta * E of one row (lane), E as 4 x 8 bf16 per plane
+            auto combine_bf16 = [&](const uint32_t (&r)[32], const uint4 (&eh)[4], const uint4 (&el)[4], float (&v)[32]) {
 #pragma unroll
-                for (int g = 0; g < 8; ++g) ew[g] = make_uint4(0, 0, 0, 0);
-                if (!need) return;
-                if (e_f32) {
-                    const float* e0 = static_cast<const float*>(P.E[0]) + row_base + col0;
+                for (int g = 0; g < 4; ++g) {
+                    const uint32_t hw[4] = {eh[g].x, eh[g].y, eh[g].z, eh[g].w};
+                    const uint32_t lw[4] = {el[g].x, el[g].y, el[g].z, el[g].w};
 #pragma unroll
-                    for (int g = 0; g < 8; ++g)
-                        if (col0 + 4 * g < P.N) ew[g] = __ldg(reinterpret_cast<const uint4*>(e0 + 4 * g));
-                } else {
-                    const __nv_bfloat16* e0 = static_cast<const __nv_bfloat16*>(P.E[0]) + row_base + col0;
-                    const __nv_bfloat16* e1 = static_cast<const __nv_bfloat16*>(P.E[1]) + row_base + col0;
+                    for (int h = 0; h < 4; ++h) {
+                        const float e0 = bf16_lo_to_f32(hw[h]) + bf16_lo_to_f32(lw[h]);
+                        const float e1 = bf16_hi_to_f32(hw[h]) + bf16_hi_to_f32(lw[h]);
+                        v[8 * g + 2 * h] = fmaf(beta, e0, alpha * __uint_as_float(r[8 * g + 2 * h]));
+                        v[8 * g + 2 * h + 1] = fmaf(beta, e1, alpha * __uint_as_float(r[8 * g + 2 * h + 1]));
+                    }
+                }
+            };
+            // Mirror store of a symmetric output, per lane: element (row, col) with col > row
+            // also goes to (col, row); for a fixed col the 32 lanes write 32 consecutive rows.
+            auto mirror_per_lane = [&](int col0, const float (&v)[32]) {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        if (col0 + 8 * g < P.N) {
-                            ew[g] = __ldg(reinterpret_cast<const uint4*>(e0 + 8 * g));
-                            if (e_lo) ew[4 + g] = __ldg(reinterpret_cast<const uint4*>(e1 + 8 * g));
+                for (int j = 0; j < 32; ++j) {
+                    const int col = col0 + j;
+                    if (row_ok && col > row && col < P.N) {
+                        const size_t off = static_cast<size_t>(col) * P.ld + row;
+                        if (out_f32) {
+                            static_cast<float*>(P.out[0])[off] = v[j];
+                        } else {
+                            const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
+                            static_cast<__nv_bfloat16*>(P.out[0])[off] = hv;
+                            if (lo_out)
+                                static_cast<__nv_bfloat16*>(P.out[1])[off] = __float2bfloat16_rn(v[j] - __bfloat162float(hv));
                         }
                     }
                 }
             };
-            uint4 ew[8];
-            load_e(c_beg, ew);
-            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status)) break;
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + acc * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
-#pragma unroll 1
-            for (int c = c_beg; c < c_end; ++c) {
-                const int col0 = ti.n0 + c * 32;
-                if (col0 >= P.N) break;  // uniform across the warp
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(t_row + c * 32, r);
-                uint4 nw[8];
-                if (c + 1 < c_end) load_e(c + 1, nw);
-                tmem_ld_wait();
-                // Rows whose whole chunk lies below the diagonal store nothing.
-                const bool any_store = row_ok && (!sym || col0 + 31 >= row);
-                float v[32];
-                if (e_f32) {
+            // Direct store of row `row` (per lane), upper triangle only for symmetric outputs.
+            auto direct_per_lane = [&](int col0, float (&v)[32]) {
+                if (!(row_ok && (!sym || col0 + 31 >= row))) return;
+                if (out_f32) {
+                    float* o = static_cast<float*>(P.out[0]) + row_base;
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
-                        const uint32_t w4[4] = {ew[g].x, ew[g].y, ew[g].z, ew[g].w};
+                        const int cg = col0 + 4 * g;
+                        if (cg >= P.N) continue;
+                        if (!sym || cg >= row) {
+                            *reinterpret_cast<float4*>(o + cg) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                        } else if (cg + 3 >= row) {
 #pragma unroll
-                        for (int h = 0; h < 4; ++h)
-                            v[4 * g + h] = fmaf(beta, __uint_as_float(w4[h]), alpha * __uint_as_float(r[4 * g + h]));
+                            for (int j = 0; j < 4; ++j)
+                                if (cg + j >= row) o[cg + j] = v[4 * g + j];
+                        }
                     }
                 } else {
+                    __nv_bfloat16* o0 = static_cast<__nv_bfloat16*>(P.out[0]) + row_base;
+                    __nv_bfloat16* o1 = static_cast<__nv_bfloat16*>(P.out[1]) + row_base;
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        const uint32_t hw[4] = {ew[g].x, ew[g].y, ew[g].z, ew[g].w};
-                        const uint32_t lw[4] = {ew[4 + g].x, ew[4 + g].y, ew[4 + g].z, ew[4 + g].w};
+                        const int cg = col0 + 8 * g;
+                        if (cg >= P.N) continue;
+                        float lo[8];
 #pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const float e0 = bf16_lo_to_f32(hw[h]) + bf16_lo_to_f32(lw[h]);
-                            const float e1 = bf16_hi_to_f32(hw[h]) + bf16_hi_to_f32(lw[h]);
-                            v[8 * g + 2 * h] = fmaf(beta, e0, alpha * __uint_as_float(r[8 * g + 2 * h]));
-                            v[8 * g + 2 * h + 1] = fmaf(beta, e1, alpha * __uint_as_float(r[8 * g + 2 * h + 1]));
-                        }
-                    }
-                }
-                if (any_store) {
-                    if (out_f32) {
-                        float* o = static_cast<float*>(P.out[0]) + row_base;
+                        for (int j = 0; j < 8; ++j)
+                            lo[j] = v[8 * g + j] - __bfloat162float(__float2bfloat16_rn(v[8 * g + j]));
+                        if (!sym || cg >= row) {
+                            store_bf16x8(o0 + cg, v + 8 * g);
+                            if (lo_out) store_bf16x8(o1 + cg, lo);
+                        } else if (cg + 7 >= row) {
 #pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            const int cg = col0 + 4 * g;
-                            if (cg >= P.N) continue;
-                            if (!sym || cg >= row) {
-                                *reinterpret_cast<float4*>(o + cg) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-                            } else if (cg + 3 >= row) {
-#pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    if (cg + j >= row) o[cg + j] = v[4 * g + j];
-                            }
-                        }
-                    } else {
-                        __nv_bfloat16* o0 = static_cast<__nv_bfloat16*>(P.out[0]) + row_base;
-                        __nv_bfloat16* o1 = static_cast<__nv_bfloat16*>(P.out[1]) + row_base;
-#pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const int cg = col0 + 8 * g;
-                            if (cg >= P.N) continue;
-                            float lo[8];
-#pragma unroll
-                            for (int j = 0; j < 8; ++j)
-                                lo[j] = v[8 * g + j] - __bfloat162float(__float2bfloat16_rn(v[8 * g + j]));
-                            if (!sym || cg >= row) {
-                                store_bf16x8(o0 + cg, v + 8 * g);
-                                if (lo_out) store_bf16x8(o1 + cg, lo);
-                            } else if (cg + 7 >= row) {
-#pragma unroll
-                                for (int j = 0; j < 8; ++j) {
-                                    if (cg + j >= row) {
-                                        o0[cg + j] = __float2bfloat16_rn(v[8 * g + j]);
-                                        if (lo_out) o1[cg + j] = __float2bfloat16_rn(lo[j]);
-                                    }
+                            for (int j = 0; j < 8; ++j) {
+                                if (cg + j >= row) {
+                                    o0[cg + j] = __float2bfloat16_rn(v[8 * g + j]);
+                                    if (lo_out) o1[cg + j] = __float2bfloat16_rn(lo[j]);
                                 }
                             }
                         }
                     }
                 }
-                if (sym) {
-                    // Mirror: element (row, col) with col > row also goes to (col, row).  For a
-                    // fixed col the 32 lanes write 32 consecutive rows: one contiguous segment.
+            };
+
+            if (!out_f32 && !e_f32) {
+                // ---------------- bf16 E and output: coalesced accesses through the staging buffers
+                // Plane 0 of E for chunk c goes by cp.async (16 bytes per lane: rows crow + 8i,
+                // segment cseg; zero-filled outside the matrix) into staging slot c & 1, one
+                // commit group per chunk, so it is in flight while the previous chunk is processed.
+                auto prefetch_e = [&](int c) {
+                    const int col0 = ti.n0 + c * 32;
+                    // chunks entirely below the diagonal of a symmetric output store nothing
+                    if (has_e && col0 < P.N && !(sym && col0 + 31 < row0)) {
+                        const __nv_bfloat16* e = static_cast<const __nv_bfloat16*>(P.E[0]);
+                        uint8_t* dst = stg_e + (c & 1) * STG_BYTES;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int col = col0 + j;
-                        if (row_ok && col > row && col < P.N) {
-                            const size_t off = static_cast<size_t>(col) * P.ld + row;
-                            if (out_f32) {
-                                static_cast<float*>(P.out[0])[off] = v[j];
-                            } else {
-                                const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
-                                static_cast<__nv_bfloat16*>(P.out[0])[off] = hv;
-                                if (lo_out)
-                                    static_cast<__nv_bfloat16*>(P.out[1])[off] = __float2bfloat16_rn(v[j] - __bfloat162float(hv));
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = row0 + crow + 8 * i;
+                            const bool in = rr < P.M;
+                            const __nv_bfloat16* src = in ? e + static_cast<size_t>(rr) * P.ld + col0 + 8 * cseg : e;
+                            cp_async16_zfill(dst + stg_off64(crow + 8 * i, cseg), src, in ? 16 : 0);
+                        }
+                    }
+                    cp_async_commit();
+                };
+                // a split E's plane 1 for chunk c, read directly (coalesced) and turned into rows
+                auto load_e_lo = [&](int c, uint4 (&el)[4]) {
+                    const int col0 = ti.n0 + c * 32;
+                    const __nv_bfloat16* e = static_cast<const __nv_bfloat16*>(P.E[1]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = row0 + crow + 8 * i;
+                        el[i] = rr < P.M ? __ldg(reinterpret_cast<const uint4*>(e + static_cast<size_t>(rr) * P.ld + col0 + 8 * cseg))
+                                         : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(stg + stg_off64(crow + 8 * i, cseg)) = el[i];
+                    __syncwarp();
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) el[g] = *reinterpret_cast<const uint4*>(stg + stg_off64(lane, g));
+                    __syncwarp();
+                };
+                prefetch_e(c_beg);
+                // the chunk loop synchronises the warp: every lane takes the same decision
+                if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status))) {
+                    cp_async_wait_all();
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = c_beg; c < c_end; ++c) {
+                    const int col0 = ti.n0 + c * 32;
+                    if (col0 >= P.N) break;  // uniform across the warp
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r);
+                    if (c + 1 < c_end) prefetch_e(c + 1);
+                    else cp_async_commit();
+                    tmem_ld_wait();
+                    // the chunk against the diagonal (uniform): rows row0 .. row0 + 31, columns
+                    // col0 .. col0 + 31, both multiples of 32
+                    const bool below = sym && col0 < row0;
+                    const bool diag = sym && col0 == row0;
+                    uint4 eh[4], el[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) { eh[i] = make_uint4(0, 0, 0, 0); el[i] = make_uint4(0, 0, 0, 0); }
+                    cp_async_wait_group<1>();   // this lane's copies of chunk c have landed
+                    __syncwarp();               // ... and every lane's
+                    if (has_e && !below) {
+                        const uint8_t* src = stg_e + (c & 1) * STG_BYTES;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) eh[g] = *reinterpret_cast<const uint4*>(src + stg_off64(lane, g));
+                        if (e_lo) load_e_lo(c, el);
+                    }
+                    __syncwarp();               // slot c & 1 is free for chunk c + 2
+                    float v[32];
+                    combine_bf16(r, eh, el, v);
+                    if (diag) {
+                        direct_per_lane(col0, v);
+                        mirror_per_lane(col0, v);
+                    } else if (!below) {
+                        // direct store (hi, then lo): per-lane rows -> staging -> 8 rows x 64 B
+                        // per instruction.  N is a multiple of 8: a 16-byte segment is wholly
+                        // inside or outside the matrix.
+#pragma unroll 1
+                        for (int pl = 0; pl < (lo_out ? 2 : 1); ++pl) {
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                float w[8];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const float x = v[8 * g + j];
+                                    w[j] = pl == 0 ? x : x - __bfloat162float(__float2bfloat16_rn(x));
+                                }
+                                uint4 pk;
+                                pk.x = pack_bf16x2(w[0], w[1]); pk.y = pack_bf16x2(w[2], w[3]);
+                                pk.z = pack_bf16x2(w[4], w[5]); pk.w = pack_bf16x2(w[6], w[7]);
+                                *reinterpret_cast<uint4*>(stg + stg_off64(lane, g)) = pk;
+                            }
+                            __syncwarp();
+                            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out[pl]);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int rr = row0 + crow + 8 * i;
+                                const int cc = col0 + 8 * cseg;
+                                const uint4 val = *reinterpret_cast<const uint4*>(stg + stg_off64(crow + 8 * i, cseg));
+                                if (rr < P.M && cc < P.N)
+                                    *reinterpret_cast<uint4*>(o + static_cast<size_t>(rr) * P.ld + cc) = val;
+                            }
+                            __syncwarp();
+                        }
+                        if (sym) {
+                            // mirror: lane L writes column L of the transposed chunk, which then
+                            // leaves as 8 rows x 64 B per instruction
+#pragma unroll 1
+                            for (int pl = 0; pl < (lo_out ? 2 : 1); ++pl) {
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
+                                    const __nv_bfloat16 bv =
+                                        pl == 0 ? hv : __float2bfloat16_rn(v[j] - __bfloat162float(hv));
+                                    *reinterpret_cast<__nv_bfloat16*>(stg_t + stg_off64(j, lane >> 3) + 2 * (lane & 7)) = bv;
+                                }
+                                __syncwarp();
+                                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out[pl]);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const int rr = col0 + crow + 8 * i;     // mirrored row
+                                    const int cc = row0 + 8 * cseg;         // mirrored columns
+                                    const uint4 val = *reinterpret_cast<const uint4*>(stg_t + stg_off64(crow + 8 * i, cseg));
+                                    if (rr < P.N && cc < P.M)
+                                        *reinterpret_cast<uint4*>(o + static_cast<size_t>(rr) * P.ld + cc) = val;
+                                }
+                                __syncwarp();
                             }
                         }
                     }
                 }
+                cp_async_wait_all();   // the trailing (empty) groups: nothing is left in flight
+            } else {
+                // ---------------- fp32 E or output: per-lane rows
+                // E of chunk c for this row: bf16 -> ew[0..3] plane 0, ew[4..7] plane 1; fp32 -> ew[0..7]
+                auto load_e = [&](int c, uint4 (&ew)[8]) {
+                    const int col0 = ti.n0 + c * 32;
+                    const bool need = has_e && row_ok && col0 < P.N && (!sym || col0 + 31 >= row);
 #pragma unroll
-                for (int g = 0; g < 8; ++g) ew[g] = nw[g];
+                    for (int g = 0; g < 8; ++g) ew[g] = make_uint4(0, 0, 0, 0);
+                    if (!need) return;
+                    if (e_f32) {
+                        const float* e0 = static_cast<const float*>(P.E[0]) + row_base + col0;
+#pragma unroll
+                        for (int g = 0; g < 8; ++g)
+                            if (col0 + 4 * g < P.N) ew[g] = __ldg(reinterpret_cast<const uint4*>(e0 + 4 * g));
+                    } else {
+                        const __nv_bfloat16* e0 = static_cast<const __nv_bfloat16*>(P.E[0]) + row_base + col0;
+                        const __nv_bfloat16* e1 = static_cast<const __nv_bfloat16*>(P.E[1]) + row_base + col0;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (col0 + 8 * g < P.N) {
+                                ew[g] = __ldg(reinterpret_cast<const uint4*>(e0 + 8 * g));
+                                if (e_lo) ew[4 + g] = __ldg(reinterpret_cast<const uint4*>(e1 + 8 * g));
+                            }
+                        }
+                    }
+                };
+                uint4 ew[8];
+                load_e(c_beg, ew);
+                if (!__all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, dev_status))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int c = c_beg; c < c_end; ++c) {
+                    const int col0 = ti.n0 + c * 32;
+                    if (col0 >= P.N) break;  // uniform across the warp
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, r);
+                    uint4 nw[8];
+                    if (c + 1 < c_end) load_e(c + 1, nw);
+                    tmem_ld_wait();
+                    float v[32];
+                    if (e_f32) {
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            const uint32_t w4[4] = {ew[g].x, ew[g].y, ew[g].z, ew[g].w};
+#pragma unroll
+                            for (int h = 0; h < 4; ++h)
+                                v[4 * g + h] = fmaf(beta, __uint_as_float(w4[h]), alpha * __uint_as_float(r[4 * g + h]));
+                        }
+                    } else {
+                        const uint4 eh[4] = {ew[0], ew[1], ew[2], ew[3]};
+                        const uint4 el[4] = {ew[4], ew[5], ew[6], ew[7]};
+                        combine_bf16(r, eh, el, v);
+                    }
+                    direct_per_lane(col0, v);
+                    if (sym) mirror_per_lane(col0, v);
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) ew[g] = nw[g];
+                }
             }
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader + acc * 8u);
             if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
     }
-
     tc_fence_before();
     cluster_sync();     // no CTA leaves while its pair may still touch its memory
     tc_fence_after();
