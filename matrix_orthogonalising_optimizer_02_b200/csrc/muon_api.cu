@@ -118,7 +118,103 @@ size_t ns_tables_bound(const std::vector<std::pair<int, int>>& shapes, const muo
 constexpr int kBoxK = kTcBM / 2, kBoxMN = 64;
 
 // ---------------------------------------------------------------- NS chain (bf16, tcgen05)
-// Appends the 3T grouped launches; returns per matrix the buffer holding the final X.
+// One stage (0 Gram, 1 polynomial, 2 apply) of iteration t for matrix m: its problem, and its
+// tiles (problem index p) appended to `tiles`.  Returns the algorithmic FLOPs.
+double ns_stage_problem(TmapPool& pool, NsMat& m, const muon_ns_schedule& sch, int t, int stage, int p,
+                        TcProblem& P, std::vector<uint32_t>& tiles, void** final_x) {
+    const int T = sch.n_iters;
+    const int cur = t & 1, nxt = cur ^ 1;
+    const bool split = t < sch.n_split_iters;
+    const bool in_lo = t > 0 && (t - 1) < sch.n_split_iters;
+    const float a = sch.coeffs[3 * t], b = sch.coeffs[3 * t + 1], c = sch.coeffs[3 * t + 2];
+    const bool last = (t == T - 1);
+    std::memset(&P, 0, sizeof(P));
+    const int r = m.r, s = m.s;
+    void* xin0 = m.X[cur][0];
+    void* xin1 = in_lo ? m.X[cur][1] : nullptr;
+    double flops = 0.0;
+    if (stage == 0) {  // A = X X^T (wide) or X^T X (tall)
+        const int box_a = m.tall ? kBoxMN : kBoxK, box_b = box_a;
+        P.tmA[0] = pool.get(xin0, m.rows, m.cols, box_a);
+        P.tmA[1] = pool.get(xin1, m.rows, m.cols, box_a);
+        P.tmB[0] = pool.get(xin0, m.rows, m.cols, box_b);
+        P.tmB[1] = pool.get(xin1, m.rows, m.cols, box_b);
+        P.out[0] = static_cast<__nv_bfloat16*>(m.A[0]);
+        P.out[1] = split ? static_cast<__nv_bfloat16*>(m.A[1]) : nullptr;
+        P.M = r; P.N = r; P.K = s; P.ld = r;
+        P.alpha = 1.f; P.beta = 0.f;
+        P.dscale = t == 0 ? m.scale : nullptr;
+        P.scale_pow = 2;
+        P.flags = kProbSym | (m.tall ? (kProbAMn | kProbBMn) : 0u);
+        flops = static_cast<double>(r) * r * s;
+    } else if (stage == 1) {  // B = b A + c A A  (A A = A A^T, A symmetric)
+        void* a1 = split ? m.A[1] : nullptr;
+        P.tmA[0] = pool.get(m.A[0], r, r, kBoxK);
+        P.tmA[1] = pool.get(a1, r, r, kBoxK);
+        P.tmB[0] = P.tmA[0];
+        P.tmB[1] = P.tmA[1];
+        P.E[0] = m.A[0];
+        P.E[1] = a1;
+        P.out[0] = static_cast<__nv_bfloat16*>(m.B[0]);
+        P.out[1] = split ? static_cast<__nv_bfloat16*>(m.B[1]) : nullptr;
+        P.M = r; P.N = r; P.K = r; P.ld = r;
+        P.alpha = c; P.beta = b;
+        P.flags = kProbSym;
+        flops = static_cast<double>(r) * r * r;
+    } else {  // X' = a X + B X (wide) or a X + X B (tall)
+        void* b1 = split ? m.B[1] : nullptr;
+        if (!m.tall) {
+            P.tmA[0] = pool.get(m.B[0], r, r, kBoxK);
+            P.tmA[1] = pool.get(b1, r, r, kBoxK);
+            P.tmB[0] = pool.get(xin0, m.rows, m.cols, kBoxMN);
+            P.tmB[1] = pool.get(xin1, m.rows, m.cols, kBoxMN);
+            P.flags = kProbBMn;
+        } else {
+            P.tmA[0] = pool.get(xin0, m.rows, m.cols, kBoxK);
+            P.tmA[1] = pool.get(xin1, m.rows, m.cols, kBoxK);
+            P.tmB[0] = pool.get(m.B[0], r, r, kBoxK);
+            P.tmB[1] = pool.get(b1, r, r, kBoxK);
+            P.flags = 0;
+        }
+        P.E[0] = xin0;
+        P.E[1] = xin1;
+        void* out0 = (last && m.final_out) ? m.final_out : m.X[nxt][0];
+        P.out[0] = static_cast<__nv_bfloat16*>(out0);
+        P.out[1] = split ? static_cast<__nv_bfloat16*>(m.X[nxt][1]) : nullptr;
+        P.M = m.rows; P.N = m.cols; P.K = r; P.ld = m.cols;
+        P.alpha = 1.f; P.beta = a;
+        P.dscale = t == 0 ? m.scale : nullptr;
+        P.scale_pow = 1;
+        flops = 2.0 * r * r * s;
+        if (last) *final_x = out0;
+    }
+    // split-bf16: hi*hi + hi*lo + lo*hi over the planes present
+    tc_set_segments(P, P.tmA[1] ? 2 : 1, P.tmB[1] ? 2 : 1, 1);
+    if (stage < 2) {
+        const int mbs = (r + kTcBM - 1) / kTcBM, nbs = (r + kTcBN - 1) / kTcBN;
+        for (int nb = 0; nb < nbs; ++nb)
+            for (int mb = 0; mb < mbs; ++mb)
+                if (kTcBN * nb + kTcBN - 1 >= kTcBM * mb) tiles.push_back(tile_code(p, mb, nb));
+    } else {
+        // Neighbouring CTA pairs (consecutive tiles) share one block of X and sweep the r x r
+        // polynomial B, which stays in L2: down the columns for a wide X (B X), along the rows
+        // for a tall X (X B).  The other order streams a tall X from DRAM once per column block.
+        const int mbs = (m.rows + kTcBM - 1) / kTcBM, nbs = (m.cols + kTcBN - 1) / kTcBN;
+        if (!m.tall) {
+            for (int nb = 0; nb < nbs; ++nb)
+                for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(p, mb, nb));
+        } else {
+            for (int mb = 0; mb < mbs; ++mb)
+                for (int nb = 0; nb < nbs; ++nb) tiles.push_back(tile_code(p, mb, nb));
+        }
+    }
+    return flops;
+}
+
+// Appends the 3T grouped launches of the chain; returns per matrix the buffer holding the
+// final X.  (Running the chain in two halves one stage apart, so that each launch paired one
+// half's Gram with the other's polynomial or apply, measured 1-3% slower on the GPT-2-small
+// set and the low-rank batch.)
 muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, const muon_ns_schedule& sch,
                         unsigned* d_status, std::vector<void*>& final_x) {
     TmapPool pool(img);
@@ -126,15 +222,9 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
     const int sms = device_sm_count();
     final_x.assign(mats.size(), nullptr);
     for (size_t i = 0; i < mats.size(); ++i) final_x[i] = mats[i].X[0][0];
-
     for (int t = 0; t < T; ++t) {
-        const int cur = t & 1, nxt = cur ^ 1;
-        const bool split = t < sch.n_split_iters;
-        const bool in_lo = t > 0 && (t - 1) < sch.n_split_iters;
-        const float a = sch.coeffs[3 * t], b = sch.coeffs[3 * t + 1], c = sch.coeffs[3 * t + 2];
-        const bool last = (t == T - 1);
         for (int stage = 0; stage < 3; ++stage) {
-            // LPT: problems with the longest K first.
+            // LPT: problems with the longest K first
             std::vector<int> order(mats.size());
             for (size_t i = 0; i < mats.size(); ++i) order[i] = static_cast<int>(i);
             auto kdim = [&](int i) { return stage == 0 ? mats[i].s : mats[i].r; };
@@ -142,91 +232,11 @@ muon_status build_ns_tc(Plan& plan, TableImage& img, std::vector<NsMat>& mats, c
             std::vector<TcProblem> probs;
             std::vector<uint32_t> tiles;
             double flops = 0.0;
-            for (int pi = 0; pi < static_cast<int>(order.size()); ++pi) {
-                NsMat& m = mats[order[pi]];
+            for (int i : order) {
                 TcProblem P;
-                std::memset(&P, 0, sizeof(P));
-                const int r = m.r, s = m.s;
-                void* xin0 = m.X[cur][0];
-                void* xin1 = in_lo ? m.X[cur][1] : nullptr;
-                if (stage == 0) {  // A = X X^T (wide) or X^T X (tall)
-                    const int box_a = m.tall ? kBoxMN : kBoxK, box_b = box_a;
-                    P.tmA[0] = pool.get(xin0, m.rows, m.cols, box_a);
-                    P.tmA[1] = pool.get(xin1, m.rows, m.cols, box_a);
-                    P.tmB[0] = pool.get(xin0, m.rows, m.cols, box_b);
-                    P.tmB[1] = pool.get(xin1, m.rows, m.cols, box_b);
-                    P.out[0] = static_cast<__nv_bfloat16*>(m.A[0]);
-                    P.out[1] = split ? static_cast<__nv_bfloat16*>(m.A[1]) : nullptr;
-                    P.M = r; P.N = r; P.K = s; P.ld = r;
-                    P.alpha = 1.f; P.beta = 0.f;
-                    P.dscale = t == 0 ? m.scale : nullptr;
-                    P.scale_pow = 2;
-                    P.flags = kProbSym | (m.tall ? (kProbAMn | kProbBMn) : 0u);
-                    flops += static_cast<double>(r) * r * s;
-                } else if (stage == 1) {  // B = b A + c A A  (A A = A A^T, A symmetric)
-                    void* a1 = split ? m.A[1] : nullptr;
-                    P.tmA[0] = pool.get(m.A[0], r, r, kBoxK);
-                    P.tmA[1] = pool.get(a1, r, r, kBoxK);
-                    P.tmB[0] = P.tmA[0];
-                    P.tmB[1] = P.tmA[1];
-                    P.E[0] = m.A[0];
-                    P.E[1] = a1;
-                    P.out[0] = static_cast<__nv_bfloat16*>(m.B[0]);
-                    P.out[1] = split ? static_cast<__nv_bfloat16*>(m.B[1]) : nullptr;
-                    P.M = r; P.N = r; P.K = r; P.ld = r;
-                    P.alpha = c; P.beta = b;
-                    P.flags = kProbSym;
-                    flops += static_cast<double>(r) * r * r;
-                } else {  // X' = a X + B X (wide) or a X + X B (tall)
-                    void* b1 = split ? m.B[1] : nullptr;
-                    if (!m.tall) {
-                        P.tmA[0] = pool.get(m.B[0], r, r, kBoxK);
-                        P.tmA[1] = pool.get(b1, r, r, kBoxK);
-                        P.tmB[0] = pool.get(xin0, m.rows, m.cols, kBoxMN);
-                        P.tmB[1] = pool.get(xin1, m.rows, m.cols, kBoxMN);
-                        P.flags = kProbBMn;
-                    } else {
-                        P.tmA[0] = pool.get(xin0, m.rows, m.cols, kBoxK);
-                        P.tmA[1] = pool.get(xin1, m.rows, m.cols, kBoxK);
-                        P.tmB[0] = pool.get(m.B[0], r, r, kBoxK);
-                        P.tmB[1] = pool.get(b1, r, r, kBoxK);
-                        P.flags = 0;
-                    }
-                    P.E[0] = xin0;
-                    P.E[1] = xin1;
-                    void* out0 = (last && m.final_out) ? m.final_out : m.X[nxt][0];
-                    P.out[0] = static_cast<__nv_bfloat16*>(out0);
-                    P.out[1] = split ? static_cast<__nv_bfloat16*>(m.X[nxt][1]) : nullptr;
-                    P.M = m.rows; P.N = m.cols; P.K = r; P.ld = m.cols;
-                    P.alpha = 1.f; P.beta = a;
-                    P.dscale = t == 0 ? m.scale : nullptr;
-                    P.scale_pow = 1;
-                    flops += 2.0 * r * r * s;
-                    if (last) final_x[order[pi]] = out0;
-                }
-                // split-bf16: hi*hi + hi*lo + lo*hi over the planes present
-                tc_set_segments(P, P.tmA[1] ? 2 : 1, P.tmB[1] ? 2 : 1, 1);
+                flops += ns_stage_problem(pool, mats[i], sch, t, stage, static_cast<int>(probs.size()), P, tiles,
+                                          &final_x[i]);
                 probs.push_back(P);
-                const int p = static_cast<int>(probs.size()) - 1;
-                if (stage < 2) {
-                    const int mbs = (r + kTcBM - 1) / kTcBM, nbs = (r + kTcBN - 1) / kTcBN;
-                    for (int nb = 0; nb < nbs; ++nb)
-                        for (int mb = 0; mb < mbs; ++mb)
-                            if (kTcBN * nb + kTcBN - 1 >= kTcBM * mb) tiles.push_back(tile_code(p, mb, nb));
-                } else {
-                    // Neighbouring CTA pairs (consecutive tiles) share one block of X and sweep
-                    // the r x r polynomial B, which stays in L2: down the columns for a wide X
-                    // (B X), along the rows for a tall X (X B).  The other order streams a tall
-                    // X from DRAM once per column block.
-                    const int mbs = (m.rows + kTcBM - 1) / kTcBM, nbs = (m.cols + kTcBN - 1) / kTcBN;
-                    if (!m.tall) {
-                        for (int nb = 0; nb < nbs; ++nb)
-                            for (int mb = 0; mb < mbs; ++mb) tiles.push_back(tile_code(p, mb, nb));
-                    } else {
-                        for (int mb = 0; mb < mbs; ++mb)
-                            for (int nb = 0; nb < nbs; ++nb) tiles.push_back(tile_code(p, mb, nb));
-                    }
-                }
             }
             if (pool.failed) return MUON_ERR_CUDA;
             const size_t po = img.add(probs.data(), probs.size() * sizeof(TcProblem), kAlign);

@@ -1,4 +1,6 @@
 // Host runtime: plan cache with pinned table images, per-kind device timing, tensor maps.
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
 #include <cstdio>
 #include <mutex>
@@ -151,8 +153,18 @@ muon_status run_plan(const std::vector<uint8_t>& key_in, void* workspace, size_t
     static const char* const kind_names[MUON_KERNEL_KINDS] = {"momentum", "scale", "ns_gemm", "update",
                                                               "simt_gemm", "lu", "misc", "tc_f32",
                                                               "simt_gemm_f64"};
+    // NVTX: one range per launch, named by kernel kind, nested in one range for the call
+    // (header-only NVTX 3: free unless a profiler injects its library)
+    nvtxRangePushA("muon_b200 plan");
+    struct RangeEnd {
+        ~RangeEnd() { nvtxRangePop(); }
+    } range_end;
     for (size_t si = 0; si < plan->steps.size(); ++si) {
         const PlanStep& s = plan->steps[si];
+        nvtxRangePushA(s.kind >= 0 && s.kind < MUON_KERNEL_KINDS ? kind_names[s.kind] : "launch");
+        struct LaunchRangeEnd {
+            ~LaunchRangeEnd() { nvtxRangePop(); }
+        } launch_range_end;
         if (g_timing.enabled) {
             TimingRec r{s.kind, s.work, nullptr, nullptr};
             cudaEventCreate(&r.e0);
