@@ -101,6 +101,10 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+    // Programmatic dependent launch: the next launch of the chain may be scheduled as this
+    // grid's CTAs finish (its prologue then overlaps this grid's tail).  It reads and writes
+    // global data only after its own grid-dependency wait below.
+    griddep_launch_dependents();
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();   // 0 = leader, 1 = peer
@@ -132,6 +136,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
 
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------------------ TMA producer
+        griddep_wait();   // operands written by the previous launch are complete and visible
         uint32_t stage = 0, phase = 0;
         int last_p = -1;
         bool ok = true;
@@ -265,6 +270,7 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
         uint8_t* stg_t = stg + STG_BYTES;              // transposed chunk of a mirror store
         uint8_t* stg_e = stg + 2 * STG_BYTES;          // E of two chunks (double buffer)
         const int crow = lane >> 2, cseg = lane & 3;   // coalesced layout: rows crow + 8i, segment cseg
+        griddep_wait();   // E, the scale and the outputs' previous readers are done
         uint32_t acc = 0, acc_phase = 0;
         for (int t = pair; t < num_tiles; t += npairs) {
             const TileInfo ti = decode(tiles[t]);
@@ -609,7 +615,20 @@ cudaError_t tc_gemm_launch(const TcProblem* d_probs, const uint32_t* d_tiles, in
         max_pairs = clusters;
     }
     const int pairs = num_tiles < max_pairs ? num_tiles : max_pairs;
-    tc_gemm_kernel<<<2 * pairs, kTcThreads, SMEM_TOTAL, stream>>>(d_probs, d_tiles, num_tiles, d_status);
+    // The grid is at most the resident capacity (every CTA runs from the start), so CTAs of the
+    // next launch that wait on this grid only take SMs that finished CTAs released.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_TOTAL;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_kernel, d_probs, d_tiles, num_tiles, d_status);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
