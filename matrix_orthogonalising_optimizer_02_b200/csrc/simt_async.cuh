@@ -19,4 +19,13 @@ bool simt_async_suits(const std::vector<SimtProblem>& probs, bool* a_kc);
 cudaError_t simt_gemm_async_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles,
                                    cudaStream_t stream, bool a_kc);
 
+// True if every problem suits dmma_gemm_launch: A, B, out (and E if used) fp64, A row-major
+// along K, B row-major along N, not symmetric, K and N even, 16-byte aligned bases and even
+// row pitches.
+bool dmma_gemm_suits(const std::vector<SimtProblem>& probs);
+
+// The same problems and 128 x 128 tile codes as simt_gemm_launch with fp64 accumulation, on
+// the double-precision tensor cores (mma.sync m16n8k4 f64).
+cudaError_t dmma_gemm_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles, cudaStream_t stream);
+
 }  // namespace muon

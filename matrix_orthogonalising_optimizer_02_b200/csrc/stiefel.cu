@@ -563,7 +563,9 @@ void add_gemm(Plan& plan, TableImage& img, const std::vector<SimtProblem>& all, 
         const int nt = static_cast<int>(tiles.size());
         bool a_kc = false;
         const bool async = !f64_acc && simt_async_suits(probs, &a_kc);
+        const bool dmma = f64_acc && dmma_gemm_suits(probs);
         plan.steps.push_back({f64_acc ? MUON_KERNEL_SIMT_GEMM_F64 : MUON_KERNEL_SIMT_GEMM, flops, [=](cudaStream_t s) {
+                                  if (dmma) return dmma_gemm_launch(dp, dt, nt, s);
                                   return async ? simt_gemm_async_launch(dp, dt, nt, s, a_kc)
                                                : simt_gemm_launch(dp, dt, nt, s, f64_acc);
                               }});
