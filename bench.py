@@ -303,22 +303,22 @@ def _stiefel(gen):
     kinds = {k: mb.timing_read(k) for k in ("tc_f32", "simt_gemm", "simt_gemm_f64", "lu", "misc")}
     work = sum(kinds[k][2] for k in ("tc_f32", "simt_gemm", "simt_gemm_f64", "lu"))
     ms = _time_ms(lambda: mb.stiefel_cayley_step(W, G, 1e-2, ws), 1, 3)
-    # ALU rooflines, one per arithmetic type, from the unit counts at the maximum SM clock
-    # (1965 MHz): 148 SMs x 128 fp32 FMA lanes x 2 FLOP = 74.4 TFLOP/s for the fp32 products,
-    # 148 SMs x 64 fp64 FMA lanes x 2 FLOP = 37.2 TFLOP/s for the fp64 LU and back-substitution
-    # updates
+    # Rooflines, one per arithmetic type, from the unit counts at the maximum SM clock
+    # (1965 MHz): 148 SMs x 128 fp32 FMA lanes x 2 FLOP = 74.4 TFLOP/s for the fp32 products;
+    # 148 SMs x 64 fp64 lanes x 2 FLOP = 37.2 TFLOP/s for the fp64 LU and back-substitution
+    # updates, which run on the fp64 tensor cores (the same peak as the fp64 FMA pipes here)
     def roof(kind, lanes, what):
         kms, _, kwork = kinds[kind]
         peak = 148 * lanes * 2 * 1.965e9 / 1e12
         ach = kwork / max(kms * 1e-3, 1e-12) / 1e12
-        return {"bound": "alu", "kernel": what, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "kernel_ms_per_step": kms,
-                "peak_source": f"148 SMs x {lanes} FMA lanes x 2 x 1965 MHz"}
+        return {"bound": "alu" if lanes == 128 else "tensor", "kernel": what, "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "kernel_ms_per_step": kms,
+                "peak_source": f"148 SMs x {lanes} lanes x 2 FLOP x 1965 MHz"}
     out["stiefel_16x4096x1024_step"] = {"ms": ms, "fma_tflops": work / (ms * 1e-3) / 1e12,
                                         "kernel_ms": {k: v[0] for k, v in kinds.items()},
                                         "tc_f32_tflops": kinds["tc_f32"][2] / max(kinds["tc_f32"][0] * 1e-3, 1e-12) / 1e12,
                                         "roofline_fp32": roof("simt_gemm", 128, "simt_gemm kernels, fp32 FMA products"),
-                                        "roofline_fp64": roof("simt_gemm_f64", 64, "simt_gemm_kernel<double>, fp64 FMA LU updates")}
+                                        "roofline_fp64": roof("simt_gemm_f64", 64, "dmma_gemm_kernel, fp64 tensor-core LU and back-substitution updates")}
     return out
 
 
