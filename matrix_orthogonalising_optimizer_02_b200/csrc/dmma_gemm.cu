@@ -6,8 +6,12 @@
 //
 // 256 threads = 8 warps in a 2 (M) x 4 (N) grid, each warp 64 x 32 = 4 x 4 tiles of 16 x 8.
 // Operand tiles go global -> shared by cp.async in 16-byte chunks (zero-filled outside the
-// matrices) through a 3-stage ring of K-steps of 16.  Shared pitches are chosen so that
-// every fragment load of a warp touches each bank group once per 16 lanes:
+// matrices) through a 3-stage ring of K-steps of 16.  The first stages of a CTA's next tile
+// are issued before the epilogue of the current one, so their latency hides behind it, and
+// the epilogue reads a half tile of E before it stores any result: E may be the output itself,
+// so loads placed after stores would each wait out a full memory latency (the LU's K = 128
+// updates spend about as long in the epilogue as in the MMAs).  Shared pitches are chosen so
+// that every fragment load of a warp touches each bank group once per 16 lanes:
 //   A as [m][k], 20 doubles per row (160 B: rows of a quarter-warp land 32 B apart mod 128),
 //   B as [k][n], 132 doubles per row (1056 B = 32 B mod 128).
 #include <cuda_runtime.h>
@@ -66,6 +70,59 @@ __device__ __forceinline__ void load_stage(const SimtProblem& P, double* As, dou
     }
 }
 
+// out = f * (alpha * acc + beta * E) for the rows of register-block rows i0, i0 + 1 of this
+// thread (two consecutive columns per access).  All E values are loaded before the first
+// store: E is either the output itself (the same element read and written by this thread)
+// or a disjoint array.
+__device__ __forceinline__ void store_half(const SimtProblem& P, const double (&acc)[4][4][4], int i0, int m_base,
+                                           int n_base, int g, int t, double alpha, double beta, bool has_e) {
+    double* O = static_cast<double*>(P.out);
+    const double* E = static_cast<const double*>(P.E);
+    double2 e[2][2][4];
+#pragma unroll
+    for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int m = m_base + 16 * (i0 + ii) + g + 8 * h, n = n_base + 8 * j + 2 * t;
+                e[ii][h][j] = (has_e && m < P.M && n < P.N)
+                                  ? *reinterpret_cast<const double2*>(E + static_cast<long long>(m) * P.ld_e + n)
+                                  : make_double2(0.0, 0.0);
+            }
+#pragma unroll
+    for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int m = m_base + 16 * (i0 + ii) + g + 8 * h;
+            if (m >= P.M) continue;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int n = n_base + 8 * j + 2 * t;
+                if (n >= P.N) continue;
+                const double v0 = fma(beta, e[ii][h][j].x, alpha * acc[i0 + ii][j][2 * h]);
+                const double v1 = fma(beta, e[ii][h][j].y, alpha * acc[i0 + ii][j][2 * h + 1]);
+                *reinterpret_cast<double2*>(O + static_cast<long long>(m) * P.ld_out + n) = make_double2(v0, v1);
+            }
+        }
+}
+
+__device__ __forceinline__ void decode_tile(uint32_t code, int& p, int& m0, int& n0) {
+    p = static_cast<int>(code >> 20);
+    m0 = static_cast<int>((code >> 10) & 1023u) * BM;
+    n0 = static_cast<int>(code & 1023u) * BN;
+}
+
+// The first STAGES - 1 K-steps of a tile, one commit group each (empty past the end).
+__device__ __forceinline__ void prologue(const SimtProblem& P, double* As, double* Bs, int m0, int n0, int tid) {
+    const int ksteps = (P.K + BKD - 1) / BKD;
+#pragma unroll
+    for (int s = 0; s < STAGES - 1; ++s) {
+        if (s < ksteps) load_stage(P, As + s * A_ELEMS, Bs + s * B_ELEMS, m0, n0, s * BKD, tid);
+        commit();
+    }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 dmma_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restrict__ tiles, int num_tiles) {
     extern __shared__ __align__(16) double smem[];
@@ -74,11 +131,13 @@ dmma_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int wm = (warp >> 2) * 64, wn = (warp & 3) * 32;   // warp tile origin in the CTA tile
-    for (int tt = blockIdx.x; tt < num_tiles; tt += gridDim.x) {
-        const uint32_t code = tiles[tt];
-        const SimtProblem& P = probs[code >> 20];
-        const int m0 = static_cast<int>((code >> 10) & 1023u) * BM;
-        const int n0 = static_cast<int>(code & 1023u) * BN;
+    int tt = blockIdx.x;
+    if (tt >= num_tiles) return;
+    int p, m0, n0;
+    decode_tile(tiles[tt], p, m0, n0);
+    prologue(probs[p], As, Bs, m0, n0, tid);
+    while (true) {
+        const SimtProblem& P = probs[p];
         double acc[4][4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -87,12 +146,6 @@ dmma_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
 #pragma unroll
                 for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.0;
         const int ksteps = (P.K + BKD - 1) / BKD;
-        __syncthreads();   // every thread is done reading the ring for the previous tile
-#pragma unroll
-        for (int s = 0; s < STAGES - 1; ++s) {
-            if (s < ksteps) load_stage(P, As + s * A_ELEMS, Bs + s * B_ELEMS, m0, n0, s * BKD, tid);
-            commit();
-        }
         for (int ks = 0; ks < ksteps; ++ks) {
             wait_group<STAGES - 2>();   // stage ks has landed (this thread's copies)
             __syncthreads();            // ... every thread's; slot (ks - 1) % STAGES is free
@@ -117,8 +170,15 @@ dmma_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
                     for (int j = 0; j < 4; ++j) dmma(acc[i][j], af[i][0], af[i][1], bf[j]);
             }
         }
-        wait_group<0>();
-        // out = f * (alpha * acc + beta * E), two consecutive columns per access
+        // every thread is done reading the ring: start the next tile's loads, then run this
+        // tile's epilogue while they land
+        __syncthreads();
+        const int next = tt + static_cast<int>(gridDim.x);
+        int np = 0, nm0 = 0, nn0 = 0;
+        if (next < num_tiles) {
+            decode_tile(tiles[next], np, nm0, nn0);
+            prologue(probs[np], As, Bs, nm0, nn0, tid);
+        }
         float f = 1.f;
         if (P.dscale != nullptr && P.scale_pow > 0) {
             const float sc = __ldg(P.dscale);
@@ -126,29 +186,12 @@ dmma_gemm_kernel(const SimtProblem* __restrict__ probs, const uint32_t* __restri
         }
         const double alpha = static_cast<double>(P.alpha * f), beta = static_cast<double>(P.beta * f);
         const bool has_e = P.beta * f != 0.f && P.E != nullptr;
-        double* O = static_cast<double*>(P.out);
-        const double* E = static_cast<const double*>(P.E);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int m = m0 + wm + 16 * i + g + 8 * h;
-                if (m >= P.M) continue;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int n = n0 + wn + 8 * j + 2 * t;
-                    if (n >= P.N) continue;
-                    double v0 = alpha * acc[i][j][2 * h], v1 = alpha * acc[i][j][2 * h + 1];
-                    if (has_e) {
-                        const double2 e = *reinterpret_cast<const double2*>(E + static_cast<long long>(m) * P.ld_e + n);
-                        v0 = fma(beta, e.x, v0);
-                        v1 = fma(beta, e.y, v1);
-                    }
-                    *reinterpret_cast<double2*>(O + static_cast<long long>(m) * P.ld_out + n) = make_double2(v0, v1);
-                }
-            }
-        }
+        store_half(P, acc, 0, m0 + wm, n0 + wn, g, t, alpha, beta, has_e);
+        store_half(P, acc, 2, m0 + wm, n0 + wn, g, t, alpha, beta, has_e);
+        if (next >= num_tiles) break;
+        tt = next; p = np; m0 = nm0; n0 = nn0;
     }
+    wait_group<0>();
 }
 
 }  // namespace

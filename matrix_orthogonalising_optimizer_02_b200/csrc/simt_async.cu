@@ -179,6 +179,58 @@ __device__ __forceinline__ void store_tile(const SimtProblem& P, const Acc (&acc
     const Acc* E = static_cast<const Acc*>(P.E);
     const bool vec = !P.sym && (reinterpret_cast<uintptr_t>(O) & 15u) == 0 && P.ld_out % V == 0 &&
                      (!has_e || ((reinterpret_cast<uintptr_t>(E) & 15u) == 0 && P.ld_e % V == 0));
+    if constexpr (sizeof(Acc) == sizeof(float)) {
+        if (vec) {
+            // Four rows at a time, every E load issued before the first store: E is either the
+            // output itself (each element read and written by this thread) or a disjoint array,
+            // and loads placed after stores would each wait out a full memory latency.
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float4 e[4][NG];
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    const int m = m0 + row_of(ty, 4 * half + ii);
+#pragma unroll
+                    for (int g = 0; g < NG; ++g) {
+                        const int nq = n0 + col_of<Acc>(tx, GW * g);
+                        e[ii][g] = (has_e && m < P.M && nq + GW - 1 < P.N)
+                                       ? *reinterpret_cast<const float4*>(E + static_cast<long long>(m) * P.ld_e + nq)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+#pragma unroll
+                for (int ii = 0; ii < 4; ++ii) {
+                    const int i = 4 * half + ii;
+                    const int m = m0 + row_of(ty, i);
+                    if (m >= P.M) continue;
+#pragma unroll
+                    for (int g = 0; g < NG; ++g) {
+                        const int nq = n0 + col_of<Acc>(tx, GW * g);
+                        if (nq >= P.N) continue;
+                        const long long oo = static_cast<long long>(m) * P.ld_out + nq;
+                        if (nq + GW - 1 < P.N) {
+                            float4 v;
+                            v.x = fmaf(beta, e[ii][g].x, alpha * acc[i][GW * g]);
+                            v.y = fmaf(beta, e[ii][g].y, alpha * acc[i][GW * g + 1]);
+                            v.z = fmaf(beta, e[ii][g].z, alpha * acc[i][GW * g + 2]);
+                            v.w = fmaf(beta, e[ii][g].w, alpha * acc[i][GW * g + 3]);
+                            *reinterpret_cast<float4*>(O + oo) = v;
+                        } else {
+                            const long long eo = static_cast<long long>(m) * P.ld_e + nq;
+#pragma unroll
+                            for (int j = 0; j < GW; ++j) {
+                                if (nq + j >= P.N) continue;
+                                Acc w = alpha * acc[i][GW * g + j];
+                                if (has_e) w = fmaf(beta, E[eo + j], w);
+                                O[oo + j] = w;
+                            }
+                        }
+                    }
+                }
+            }
+            return;
+        }
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int m = m0 + row_of(ty, i);
