@@ -211,6 +211,13 @@ __global__ void block_cast_kernel(const BlockCastItem* __restrict__ items, int c
 // so the per-row sweeps are free of bank conflicts).  Records the pivot row of each column
 // in piv (absolute row indices).
 __host__ __device__ constexpr int panel_pitch(int rows) { return rows | 1; }
+// 8-byte global -> shared copy, zero-filled beyond src_bytes (0 or 8).
+__device__ __forceinline__ void cp_async8(double* smem_dst, const double* gmem_src, int src_bytes) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(d), "l"(gmem_src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __global__ void __launch_bounds__(1024)
 lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int nb, int* piv, long long piv_stride,
                 unsigned* status) {
@@ -223,10 +230,13 @@ lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int 
     const int rows = N - j0;
     const int pitch = panel_pitch(rows);
     const int tid = threadIdx.x, nt = blockDim.x;
+    // cp.async: every copy in flight at once (a register round trip per element would order
+    // each global load behind the previous shared store)
     for (int e = tid; e < rows * nb; e += nt) {
         const int r = e / nb, c = e % nb;
-        pan[c * pitch + r] = a[(j0 + static_cast<long long>(r)) * ld + j0 + c];
+        cp_async8(pan + c * pitch + r, a + (j0 + static_cast<long long>(r)) * ld + j0 + c, 8);
     }
+    cp_async_wait_all();
     __syncthreads();
     for (int jj = 0; jj < nb; ++jj) {
         const double* colj = pan + jj * pitch;
@@ -327,8 +337,10 @@ template <int R, int P>
 __device__ __forceinline__ void load_block_cols(double* T, const double* a, long long ld, int r0, int w) {
     for (int e = threadIdx.x; e < R * R; e += blockDim.x) {
         const int i = e / R, l = e % R;
-        T[l * P + i] = (i < w && l < w) ? a[(r0 + static_cast<long long>(i)) * ld + r0 + l] : 0.0;
+        const bool in = i < w && l < w;
+        cp_async8(T + l * P + i, in ? a + (r0 + static_cast<long long>(i)) * ld + r0 + l : a, in ? 8 : 0);
     }
+    cp_async_wait_all();
 }
 
 // Lane h's rows r0 + G*m + h (< r0 + w) of the column starting at p (pitch ld), zero beyond.
@@ -351,49 +363,88 @@ __device__ __forceinline__ void store_column(const double (&x)[R / G], double* p
     }
 }
 
-// Applies the row interchanges of rows r0..r0+w-1 (in order) to column c.
-__device__ __forceinline__ void apply_swaps(double* a, long long ld, const int* pv, int r0, int w, int c) {
-    for (int i = 0; i < w; ++i) {
-        const int p = pv[r0 + i];
-        if (p != r0 + i) {
-            const double t = a[(r0 + static_cast<long long>(i)) * ld + c];
-            a[(r0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
-            a[static_cast<long long>(p) * ld + c] = t;
-        }
-    }
-}
-
 // Row swaps then unit-lower solve U12 = L11^-1 A12 with the w x w triangle at (r0, r0), for
-// the columns [c_lo, ncols) -- blockDim.x / G columns per block.  The group's first lane
-// applies the swaps; every lane of a warp reaches the shuffles.
+// the columns [c_lo, ncols) -- blockDim.x / G columns per block.  The interchanges of rows
+// r0..r0+w-1 (in order) are applied as one permutation: thread 0 replays them on row indices
+// in shared memory (cur[x - r0] = the original row that ends at row x), then every column
+// gathers its w rows, and the rows below the block that receive one, with independent loads
+// before it stores anything.  (Applied swap by swap, each column's 2w loads would wait on one
+// another through the stores between them.)  iw holds nrows - r0 + 2R ints of shared memory;
+// every lane of a warp reaches the shuffles.
 template <int R, int G>
 __device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const int* pv, int r0, int w, int c_lo,
-                                                int ncols, double* T) {
+                                                int ncols, int nrows, double* T, int* iw) {
     constexpr int P = R + 2;
+    __shared__ int s_nm;
+    int* mv = iw;              // R destinations, then R sources, of rows below the block
+    int* cur = iw + 2 * R;     // nrows - r0 entries
+    for (int x = threadIdx.x; x < nrows - r0; x += blockDim.x) cur[x] = r0 + x;
+    for (int i = threadIdx.x; i < w; i += blockDim.x) mv[i] = pv[r0 + i];   // the pivots, for thread 0
     load_block_cols<R, P>(T, a, ld, r0, w);
     __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < w; ++i) {
+            const int p = mv[i];
+            if (p != r0 + i && p > r0 + i && p < nrows) {
+                const int t = cur[i];
+                cur[i] = cur[p - r0];
+                cur[p - r0] = t;
+            }
+        }
+        int nm = 0;
+        for (int i = 0; i < w; ++i) {
+            const int p = mv[i];
+            if (p >= r0 + w && p < nrows && cur[p - r0] != p) {
+                mv[R + nm] = cur[p - r0];   // source (mv[nm] below is overwritten only after mv[i] is read)
+                cur[p - r0] = p;            // recorded once
+                mv[nm] = p;
+                ++nm;
+            }
+        }
+        s_nm = nm;
+    }
+    __syncthreads();
+    const int nm = s_nm;
     const int c = c_lo + static_cast<int>(blockIdx.x * (blockDim.x / G) + threadIdx.x / G);
     const int h = static_cast<int>(threadIdx.x) % G;
     const bool live = c < ncols;
-    if (live && h == 0) apply_swaps(a, ld, pv, r0, w, c);
-    __syncwarp();
-    double* col = a + (live ? c : c_lo) + r0 * ld;
-    const int wl = live ? w : 0;
-    double x[R / G];
-    load_column<R, G>(x, col, ld, wl, h);
+    double* col = a + (live ? c : c_lo);
+    double x[R / G], y[R / G];
+#pragma unroll
+    for (int m = 0; m < R / G; ++m) {
+        const int row = G * m + h;
+        x[m] = (live && row < w) ? col[static_cast<long long>(cur[row]) * ld] : 0.0;
+        y[m] = (live && row < nm) ? col[static_cast<long long>(mv[R + row]) * ld] : 0.0;
+    }
+#pragma unroll
+    for (int m = 0; m < R / G; ++m) {
+        const int j = G * m + h;
+        if (live && j < nm) col[static_cast<long long>(mv[j]) * ld] = y[m];
+    }
     solve_unit_lower<R, G, P>(x, T, h);
-    store_column<R, G>(x, col, ld, wl, h);
+#pragma unroll
+    for (int m = 0; m < R / G; ++m) {
+        const int row = G * m + h;
+        if (live && row < w) col[(r0 + static_cast<long long>(row)) * ld] = x[m];
+    }
+}
+
+// Shared memory of swap_trsm_block beyond the triangle: 2R ints plus one per row from r0 on.
+__host__ __device__ constexpr size_t swap_ints_bytes(int R, int rows_from_r0) {
+    return (2 * static_cast<size_t>(R) + static_cast<size_t>(rows_from_r0)) * sizeof(int);
 }
 
 // For each column c in [j0 + nb, ncols): apply the panel's row swaps in order, then solve
 // the unit-lower nb x nb triangle L11 (U12 = L11^-1 A12).  nb <= kPanelMax.
 constexpr int kPanelMax = 32, kPanelLanes = 2;
+constexpr size_t kPanelTriangleBytes = static_cast<size_t>(kPanelMax) * (kPanelMax + 2) * sizeof(double);
 __global__ void __launch_bounds__(128)
 lu_swap_trsm_kernel(double* Aug, long long ld, long long stride, int j0, int nb, int ncols, const int* piv,
                     long long piv_stride) {
-    __shared__ __align__(16) double T[kPanelMax * (kPanelMax + 2)];
+    extern __shared__ __align__(16) double T[];
+    int* iw = reinterpret_cast<int*>(T + kPanelMax * (kPanelMax + 2));
     swap_trsm_block<kPanelMax, kPanelLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, j0, nb,
-                                            j0 + nb, ncols, T);
+                                            j0 + nb, ncols, static_cast<int>(piv_stride), T, iw);
 }
 
 // Within the current block column: apply the row swaps of panel rows j0..j0+w-1 to the
@@ -420,12 +471,14 @@ __global__ void lu_swap_cols_kernel(double* Aug, long long ld, long long stride,
 // columns (512 threads, 8 lanes per column).
 constexpr int kLuBlock = 128, kLuLanes = 8, kTrsmThreads = 512;
 constexpr size_t kLuTriangleBytes = static_cast<size_t>(kLuBlock) * (kLuBlock + 2) * sizeof(double);
+constexpr int kMaxAugRows = 2 * 4096;   // 2k for the largest k the entry points accept
 __global__ void __launch_bounds__(kTrsmThreads)
 lu_block_swap_trsm_kernel(double* Aug, long long ld, long long stride, int J0, int JB, int c_lo, int ncols,
                           const int* piv, long long piv_stride) {
     extern __shared__ __align__(16) double T[];
+    int* iw = reinterpret_cast<int*>(T + kLuBlock * (kLuBlock + 2));
     swap_trsm_block<kLuBlock, kLuLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, J0, JB, c_lo,
-                                        ncols, T);
+                                        ncols, static_cast<int>(piv_stride), T, iw);
 }
 
 // Back substitution on one diagonal block: rows i0..i0+bs-1 of the right-hand columns
@@ -453,10 +506,10 @@ back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, in
     store_column<kBackBlock, kBackLanes>(x, col, ld, wl, h);
 }
 
-// Widest panel (<= 32 columns) whose fp64 copy (nb columns of panel_pitch(N)) fits in 200 KB
-// of shared memory.
-int lu_panel_width(int N) {
-    const int nb = static_cast<int>((200 * 1024) / (static_cast<size_t>(panel_pitch(N)) * sizeof(double)));
+// Widest panel (<= 32 columns) whose fp64 copy (nb columns of panel_pitch(rows)) fits in
+// 200 KB of shared memory.
+int lu_panel_width(int rows) {
+    const int nb = static_cast<int>((200 * 1024) / (static_cast<size_t>(panel_pitch(rows)) * sizeof(double)));
     return std::max(1, std::min(kPanelMax, nb));
 }
 
@@ -708,7 +761,8 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
                 const int block_end = J0 + JB;
                 plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right_in * B, [=](cudaStream_t s) {
                     constexpr int cols_per_block = 128 / kPanelLanes;
-                    lu_swap_trsm_kernel<<<dim3((right_in + cols_per_block - 1) / cols_per_block, B), 128, 0, s>>>(
+                    const size_t smem = kPanelTriangleBytes + swap_ints_bytes(kPanelMax, N - j0);
+                    lu_swap_trsm_kernel<<<dim3((right_in + cols_per_block - 1) / cols_per_block, B), 128, smem, s>>>(
                         Aug, ld, aug_stride, j0, w, block_end, piv, N);
                     return cudaGetLastError();
                 }});
@@ -726,10 +780,11 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
             const int c_lo = J0 + JB;
             plan.steps.push_back({MUON_KERNEL_LU, 1.0 * JB * JB * right * B, [=](cudaStream_t s) {
                 constexpr int cols_per_block = kTrsmThreads / kLuLanes;
-                cudaError_t e = big_smem<lu_block_swap_trsm_kernel>(kLuTriangleBytes);
+                cudaError_t e = big_smem<lu_block_swap_trsm_kernel>(kLuTriangleBytes + swap_ints_bytes(kLuBlock, kMaxAugRows));
                 if (e != cudaSuccess) return e;
+                const size_t smem = kLuTriangleBytes + swap_ints_bytes(kLuBlock, N - J0);
                 lu_block_swap_trsm_kernel<<<dim3((right + cols_per_block - 1) / cols_per_block, B), kTrsmThreads,
-                                            kLuTriangleBytes, s>>>(Aug, ld, aug_stride, J0, JB, c_lo, ncols, piv, N);
+                                            smem, s>>>(Aug, ld, aug_stride, J0, JB, c_lo, ncols, piv, N);
                 return cudaGetLastError();
             }});
             if (N - J0 - JB > 0) {
@@ -951,7 +1006,6 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
     auto bm = [&](int i) { return Mat{bb + i * nk, k, false, false}; };
     auto Sm = [&](int i) { return Mat{S + i * kk, k, false, false}; };
     auto Ai = [&](int i) { return Aug + i * aug_stride; };
-    auto Am = [&](int i, long long off) { return Mat{Ai(i) + off, ld, false, true}; };
 
     std::vector<SimtProblem> pr;
     const bool tc = L.tc;
