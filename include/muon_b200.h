@@ -168,10 +168,13 @@ MUON_API muon_status ns_orthogonalize(const void* X_in, int in_dtype, void* X_ou
 
 /* Stiefel-manifold step for a contiguous batch of column-orthonormal W (n x k fp32,
  * n >= k): tangent projection of G (n x k fp32), then the Cayley retraction with
- * c = lr/2 in Woodbury form.  The direction's two products (W^T G and W sym(.)) run on the
- * tensor cores as three bf16 planes (fp32-exact operands, fp32 accumulation); every product
- * that enters the retraction runs in fp32 FMA arithmetic (no TF32); the 2k x 2k system is
- * solved by fp64 Gaussian elimination with partial pivoting.
+ * c = lr/2 in Woodbury form (§6.2), evaluated through (I + cA)^-1 (I - cA) = 2 (I + cA)^-1 - I
+ * as W - 2 U C^-1 (c B W) with U = [V, W], B = [W^T; -V^T], C = I + c B U: the same map as the
+ * page's b / y = B b steps with two n x k products fewer.  The direction's two products
+ * (W^T G and W sym(.)) run on the tensor cores as three bf16 planes (fp32-exact operands,
+ * fp32 accumulation); every product that enters the retraction runs in fp32 FMA arithmetic
+ * (no TF32); the 2k x 2k system is solved by fp64 Gaussian elimination with partial
+ * pivoting.
  * W is updated in place; G is read.  n < k returns MUON_ERR_UNSUPPORTED_SHAPE (transpose
  * the problem, as the page advises).  k <= 4096. */
 MUON_API size_t stiefel_workspace_size(int batch, int n, int k);
@@ -247,8 +250,8 @@ typedef enum {
     MUON_KERNEL_LU = 5,           /* 2k x 2k LU and triangular solves                     */
     MUON_KERNEL_MISC = 6,         /* casts, copies, block assembly, plane splits          */
     MUON_KERNEL_TC_F32 = 7,       /* tcgen05 fp32 products from three bf16 planes (Stiefel) */
-    MUON_KERNEL_SIMT_GEMM_F64 = 8,  /* fp64 DFMA GEMMs (Stiefel LU trailing updates and
-                                       back substitution)                                  */
+    MUON_KERNEL_SIMT_GEMM_F64 = 8,  /* fp64 GEMMs (Stiefel LU updates and back substitution),
+                                       on the fp64 tensor cores where the layout allows  */
     MUON_KERNEL_KINDS = 9
 } muon_kernel_kind;
 MUON_API muon_status muon_timing_enable(int enable);

@@ -3,12 +3,16 @@
 //   §6.2       Cayley retraction W <- (I + cA)^-1 (I - cA) W, A = V W^T - W V^T = U B with
 //              U = [V, W], B = [W^T; -V^T], c = lr/2, through the 2k x 2k system
 //              C = I + c B U = [[I + cP, cQ], [-cR, I - cP^T]]   (P = W^T V, Q = W^T W, R = V^T V)
-//              b = W - c U (B W) = W - c V Q + c W P^T,  y = B b = [W^T b; -V^T b]
-//              z = C^-1 y,  W_new = b - c (V z_top + W z_bot)
+//              The page's Woodbury steps (b = W - c U B W, y = B b, z = C^-1 y,
+//              W_new = b - c U z) are taken through the identity
+//              (I + cA)^-1 (I - cA) = 2 (I + cA)^-1 - I, which gives the same map with y
+//              replaced by c B W = [cQ; -cP^T] (the right block column of C - I, no product):
+//              z = C^-1 [cQ; -cP^T],  W_new = W - 2 (V z_top + W z_bot).
+//              That drops the products for b and y, half the n x k fp32 work.
 // No TF32 anywhere.  The n x k panel products run on the FMA pipes in fp32; the reductions
-// over n (W^T G, the blocks P, Q, R and y) are split into 512-row chunks accumulated in fp32
+// over n (W^T G and the blocks P, Q, R) are split into 512-row chunks accumulated in fp32
 // in parallel and summed in fp64.  The augmented 2k x (2k + k)
-// matrix [C | y] is held and eliminated in fp64 (Gaussian elimination with partial
+// matrix [C | c B W] is held and eliminated in fp64 (Gaussian elimination with partial
 // pivoting, blocked: panel factorisation in shared memory, row swaps + unit-lower solve on
 // the right-hand columns, rank-nb GEMM update), then blocked back substitution: C has
 // condition numbers around 1e3 at n = 4096, k = 1024, and an fp32 solve alone lets the
@@ -48,6 +52,17 @@ __global__ void aug_neg_transpose_kernel(double* Aug, int k, long long ld, long 
          e += static_cast<long long>(gridDim.x) * blockDim.x) {
         const int i = static_cast<int>(e / k), j = static_cast<int>(e % k);
         a[(k + static_cast<long long>(i)) * ld + k + j] = -a[static_cast<long long>(j) * ld + i];
+    }
+}
+
+// Right-hand side of the Woodbury solve: columns 2k..3k-1 <- columns k..2k-1, all 2k rows.
+__global__ void aug_copy_rhs_kernel(double* Aug, int k, long long ld, long long stride) {
+    double* a = Aug + blockIdx.y * stride;
+    const long long total = 2LL * k * k;
+    for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long i = e / k, j = e % k;
+        a[i * ld + 2LL * k + j] = a[i * ld + k + j];
     }
 }
 
@@ -372,15 +387,15 @@ __device__ __forceinline__ void store_column(const double (&x)[R / G], double* p
 // another through the stores between them.)  iw holds nrows - r0 + 2R ints of shared memory;
 // every lane of a warp reaches the shuffles.
 template <int R, int G>
-__device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const int* pv, int r0, int w, int c_lo,
-                                                int ncols, int nrows, double* T, int* iw) {
+__device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const int* pv, int r0, int w, int c_first,
+                                                int c_end, bool solve, int nrows, double* T, int* iw) {
     constexpr int P = R + 2;
     __shared__ int s_nm;
     int* mv = iw;              // R destinations, then R sources, of rows below the block
     int* cur = iw + 2 * R;     // nrows - r0 entries
     for (int x = threadIdx.x; x < nrows - r0; x += blockDim.x) cur[x] = r0 + x;
     for (int i = threadIdx.x; i < w; i += blockDim.x) mv[i] = pv[r0 + i];   // the pivots, for thread 0
-    load_block_cols<R, P>(T, a, ld, r0, w);
+    if (solve) load_block_cols<R, P>(T, a, ld, r0, w);
     __syncthreads();
     if (threadIdx.x == 0) {
         for (int i = 0; i < w; ++i) {
@@ -405,10 +420,10 @@ __device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const i
     }
     __syncthreads();
     const int nm = s_nm;
-    const int c = c_lo + static_cast<int>(blockIdx.x * (blockDim.x / G) + threadIdx.x / G);
+    const int c = c_first + static_cast<int>(threadIdx.x) / G;
     const int h = static_cast<int>(threadIdx.x) % G;
-    const bool live = c < ncols;
-    double* col = a + (live ? c : c_lo);
+    const bool live = c < c_end;
+    double* col = a + (live ? c : c_first);
     double x[R / G], y[R / G];
 #pragma unroll
     for (int m = 0; m < R / G; ++m) {
@@ -421,7 +436,7 @@ __device__ __forceinline__ void swap_trsm_block(double* a, long long ld, const i
         const int j = G * m + h;
         if (live && j < nm) col[static_cast<long long>(mv[j]) * ld] = y[m];
     }
-    solve_unit_lower<R, G, P>(x, T, h);
+    if (solve) solve_unit_lower<R, G, P>(x, T, h);   // uniform across the block
 #pragma unroll
     for (int m = 0; m < R / G; ++m) {
         const int row = G * m + h;
@@ -434,35 +449,23 @@ __host__ __device__ constexpr size_t swap_ints_bytes(int R, int rows_from_r0) {
     return (2 * static_cast<size_t>(R) + static_cast<size_t>(rows_from_r0)) * sizeof(int);
 }
 
-// For each column c in [j0 + nb, ncols): apply the panel's row swaps in order, then solve
-// the unit-lower nb x nb triangle L11 (U12 = L11^-1 A12).  nb <= kPanelMax.
-constexpr int kPanelMax = 32, kPanelLanes = 2;
+// After a panel j0..j0+nb-1 of the block column starting at c_left: the panel's row swaps,
+// applied to the block's earlier multiplier columns [c_left, j0) (blocks 0 .. left_blocks - 1)
+// and, with the solve U12 = L11^-1 A12 by the unit-lower nb x nb triangle L11, to the block's
+// columns [j0 + nb, ncols) (the remaining blocks).  nb <= kPanelMax.
+constexpr int kPanelMax = 32, kPanelLanes = 2, kPanelSwapThreads = 128;
+constexpr int kPanelSwapCols = kPanelSwapThreads / kPanelLanes;
 constexpr size_t kPanelTriangleBytes = static_cast<size_t>(kPanelMax) * (kPanelMax + 2) * sizeof(double);
-__global__ void __launch_bounds__(128)
-lu_swap_trsm_kernel(double* Aug, long long ld, long long stride, int j0, int nb, int ncols, const int* piv,
-                    long long piv_stride) {
+__global__ void __launch_bounds__(kPanelSwapThreads)
+lu_swap_trsm_kernel(double* Aug, long long ld, long long stride, int c_left, int left_blocks, int j0, int nb,
+                    int ncols, const int* piv, long long piv_stride) {
     extern __shared__ __align__(16) double T[];
     int* iw = reinterpret_cast<int*>(T + kPanelMax * (kPanelMax + 2));
+    const bool left = static_cast<int>(blockIdx.x) < left_blocks;
+    const int c_first = left ? c_left + static_cast<int>(blockIdx.x) * kPanelSwapCols
+                             : j0 + nb + (static_cast<int>(blockIdx.x) - left_blocks) * kPanelSwapCols;
     swap_trsm_block<kPanelMax, kPanelLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, j0, nb,
-                                            j0 + nb, ncols, static_cast<int>(piv_stride), T, iw);
-}
-
-// Within the current block column: apply the row swaps of panel rows j0..j0+w-1 to the
-// earlier multiplier columns [c_lo, c_hi), so the block's L stays consistently permuted.
-__global__ void lu_swap_cols_kernel(double* Aug, long long ld, long long stride, int c_lo, int c_hi, int j0, int w,
-                                    const int* piv, long long piv_stride) {
-    double* a = Aug + blockIdx.y * stride;
-    const int* pv = piv + blockIdx.y * piv_stride;
-    const int c = c_lo + blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= c_hi) return;
-    for (int i = 0; i < w; ++i) {
-        const int p = pv[j0 + i];
-        if (p != j0 + i) {
-            const double t = a[(j0 + static_cast<long long>(i)) * ld + c];
-            a[(j0 + static_cast<long long>(i)) * ld + c] = a[static_cast<long long>(p) * ld + c];
-            a[static_cast<long long>(p) * ld + c] = t;
-        }
-    }
+                                            c_first, left ? j0 : ncols, !left, static_cast<int>(piv_stride), T, iw);
 }
 
 // After a block column J0..J0+JB-1 is factorised: for every column c >= c_lo, apply the
@@ -477,8 +480,9 @@ lu_block_swap_trsm_kernel(double* Aug, long long ld, long long stride, int J0, i
                           const int* piv, long long piv_stride) {
     extern __shared__ __align__(16) double T[];
     int* iw = reinterpret_cast<int*>(T + kLuBlock * (kLuBlock + 2));
-    swap_trsm_block<kLuBlock, kLuLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, J0, JB, c_lo,
-                                        ncols, static_cast<int>(piv_stride), T, iw);
+    swap_trsm_block<kLuBlock, kLuLanes>(Aug + blockIdx.y * stride, ld, piv + blockIdx.y * piv_stride, J0, JB,
+                                        c_lo + static_cast<int>(blockIdx.x) * (kTrsmThreads / kLuLanes), ncols, true,
+                                        static_cast<int>(piv_stride), T, iw);
 }
 
 // Back substitution on one diagonal block: rows i0..i0+bs-1 of the right-hand columns
@@ -506,10 +510,12 @@ back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, in
     store_column<kBackBlock, kBackLanes>(x, col, ld, wl, h);
 }
 
-// Widest panel (<= 32 columns) whose fp64 copy (nb columns of panel_pitch(rows)) fits in
-// 200 KB of shared memory.
+// Shared memory of a panel: nb fp64 columns of panel_pitch(rows).  The widest panel (<= 32
+// columns) that fits in kPanelSmem is used.
+constexpr size_t kPanelSmem = 200 * 1024;
+size_t lu_panel_smem(int rows, int nb) { return static_cast<size_t>(panel_pitch(rows)) * nb * sizeof(double); }
 int lu_panel_width(int rows) {
-    const int nb = static_cast<int>((200 * 1024) / (static_cast<size_t>(panel_pitch(rows)) * sizeof(double)));
+    const int nb = static_cast<int>(kPanelSmem / (static_cast<size_t>(panel_pitch(rows)) * sizeof(double)));
     return std::max(1, std::min(kPanelMax, nb));
 }
 
@@ -722,15 +728,20 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
     auto Ai = [&](int i) { return Aug + i * aug_stride; };
     std::vector<SimtProblem> pr;
     // Gaussian elimination with partial pivoting on [C | y], fp64, two levels: kLuBlock-wide
-    // block columns factorised with nb-wide panels (updates confined to the block column),
-    // then one row-swap + unit-lower solve over the trailing columns and one K = kLuBlock
-    // trailing update per block column.
-    const int nb = lu_panel_width(N);
+    // block columns factorised with panels (updates confined to the block column), then one
+    // row-swap + unit-lower solve over the trailing columns and one K = kLuBlock trailing
+    // update per block column.  A panel holds its rows from the block column's top down in
+    // shared memory, so the lower block columns take wider panels (fewer, up to kPanelMax
+    // columns), split evenly across the block column.  Widths are even, so the in-block updates
+    // (K = the width, N = the block's remaining columns) suit the fp64 tensor-core kernel.
     for (int J0 = 0; J0 < N; J0 += kLuBlock) {
         const int JB = std::min(kLuBlock, N - J0);
+        const int widest = std::max(2, lu_panel_width(N - J0) & ~1);
+        const int npan = (JB + widest - 1) / widest;
+        const int nb = std::min(widest, ((JB + npan - 1) / npan + 1) & ~1);
         for (int j0 = J0; j0 < J0 + JB; j0 += nb) {
             const int w = std::min(nb, J0 + JB - j0);
-            const size_t smem = static_cast<size_t>(panel_pitch(N - j0)) * w * sizeof(double);
+            const size_t smem = lu_panel_smem(N - j0, w);
             const double lu_flops = 2.0 * (N - j0) * w * w * B;
             plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
                 // the function attribute is per device: set once on each (launches run under
@@ -741,31 +752,27 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
                 if (e != cudaSuccess) return e;
                 if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
                 if (!attr_set[dev]) {
-                    e = cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024 + 1024);
+                    e = cudaFuncSetAttribute(lu_panel_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kPanelSmem));
                     if (e != cudaSuccess) return e;
                     attr_set[dev] = true;
                 }
                 lu_panel_kernel<<<B, 1024, smem, s>>>(Aug, ld, aug_stride, N, j0, w, piv, N, d_status);
                 return cudaGetLastError();
             }});
-            if (j0 > J0) {
-                const int left = j0 - J0;
-                plan.steps.push_back({MUON_KERNEL_LU, 0.0, [=](cudaStream_t s) {
-                    lu_swap_cols_kernel<<<dim3((left + 127) / 128, B), 128, 0, s>>>(Aug, ld, aug_stride, J0, j0, j0, w,
-                                                                                    piv, N);
+            // the panel's swaps on the block's earlier columns, swaps + solve on its later ones
+            const int right_in = J0 + JB - (j0 + w);
+            const int left_blocks = (j0 - J0 + kPanelSwapCols - 1) / kPanelSwapCols;
+            const int right_blocks = (right_in + kPanelSwapCols - 1) / kPanelSwapCols;
+            if (left_blocks + right_blocks > 0) {
+                const int block_end = J0 + JB;
+                plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * std::max(right_in, 0) * B, [=](cudaStream_t s) {
+                    const size_t smem = kPanelTriangleBytes + swap_ints_bytes(kPanelMax, N - j0);
+                    lu_swap_trsm_kernel<<<dim3(left_blocks + right_blocks, B), kPanelSwapThreads, smem, s>>>(
+                        Aug, ld, aug_stride, J0, left_blocks, j0, w, block_end, piv, N);
                     return cudaGetLastError();
                 }});
             }
-            const int right_in = J0 + JB - (j0 + w);
             if (right_in > 0) {
-                const int block_end = J0 + JB;
-                plan.steps.push_back({MUON_KERNEL_LU, 1.0 * w * w * right_in * B, [=](cudaStream_t s) {
-                    constexpr int cols_per_block = 128 / kPanelLanes;
-                    const size_t smem = kPanelTriangleBytes + swap_ints_bytes(kPanelMax, N - j0);
-                    lu_swap_trsm_kernel<<<dim3((right_in + cols_per_block - 1) / cols_per_block, B), 128, smem, s>>>(
-                        Aug, ld, aug_stride, j0, w, block_end, piv, N);
-                    return cudaGetLastError();
-                }});
                 for (int i = 0; i < B; ++i) {
                     double* base = Ai(i);
                     pr.push_back(gemm(Mat{base + (j0 + w) * ld + j0, ld, false, true}, Mat{base + j0 * ld + j0 + w, ld, false, true},
@@ -1003,7 +1010,6 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
     auto Wm = [&](int i, bool t = false) { return Mat{W + i * nk, k, t, false}; };
     auto Gm = [&](int i) { return Mat{G + i * nk, k, false, false}; };
     auto Vm = [&](int i, bool t = false) { return Mat{V + i * nk, k, t, false}; };
-    auto bm = [&](int i) { return Mat{bb + i * nk, k, false, false}; };
     auto Sm = [&](int i) { return Mat{S + i * kk, k, false, false}; };
     auto Ai = [&](int i) { return Aug + i * aug_stride; };
 
@@ -1092,29 +1098,23 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
         add_block_cast(plan, img, items);
     };
     auto Bm32 = [&](int i, int which) { return Mat{blocks32(i, which), k, false, false}; };
-    // b = W - V (cQ) - W (-c P^T)
-    cast_blocks(k, k * ld + k);
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Bm32(i, 0), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -1.f, 1.f));
-    add_gemm(plan, img, pr); pr.clear();
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Bm32(i, 1), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -1.f, 1.f));
-    add_gemm(plan, img, pr); pr.clear();
+    // right-hand side [cQ; -cP^T] = c B W: the right block column of cBU, copied before the
+    // identity is added
+    plan.steps.push_back({MUON_KERNEL_MISC, 32.0 * kk * B, [=](cudaStream_t s) {
+        aug_copy_rhs_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((2 * kk + 255) / 256))), B), 256, 0, s>>>(Aug, k, ld, aug_stride);
+        return cudaGetLastError();
+    }});
     // C = I + c B U
     plan.steps.push_back({MUON_KERNEL_MISC, 16.0 * N * B, [=](cudaStream_t s) {
         aug_add_identity_kernel<<<dim3((N + 255) / 256, B), 256, 0, s>>>(Aug, N, ld, aug_stride);
         return cudaGetLastError();
     }});
-    // y = [W^T b; -V^T b] into the right-hand columns (split-K sums)
-    for (int i = 0; i < B; ++i) {
-        pr.push_back(gemm(Wm(i, true), bm(i), Ai(i) + N, ld, true, nullptr, 0, false, k, k, n, 1.f, 0.f));
-        pr.push_back(gemm(Vm(i, true), bm(i), Ai(i) + k * ld + N, ld, true, nullptr, 0, false, k, k, n, -1.f, 0.f));
-    }
-    add_gemm_splitk(plan, img, pr, part); pr.clear();
     add_lu_solve(plan, img, Aug, piv, N, ncols, k, B, ld, aug_stride, d_status);
-    // W_new = b - c V z_top - c W z_bot, then copy into W
+    // W_new = W - 2 (V z_top + W z_bot), z = C^-1 (c B W), through the workspace b, then into W
     cast_blocks(N, k * ld + N);
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Bm32(i, 0), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Vm(i), Bm32(i, 0), bb + i * nk, k, false, W + i * nk, k, false, n, k, k, -2.f, 1.f));
     add_gemm(plan, img, pr); pr.clear();
-    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Bm32(i, 1), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -c, 1.f));
+    for (int i = 0; i < B; ++i) pr.push_back(gemm(Wm(i), Bm32(i, 1), bb + i * nk, k, false, bb + i * nk, k, false, n, k, k, -2.f, 1.f));
     add_gemm(plan, img, pr); pr.clear();
     const size_t bytes = static_cast<size_t>(nk) * B * sizeof(float);
     plan.steps.push_back({MUON_KERNEL_MISC, 2.0 * bytes, [=](cudaStream_t s) {

@@ -126,3 +126,25 @@ def test_muon_cayley_wide_batch_matches_transposed_oracle():
         assert np.max(np.abs(got - Wr[i])) <= 2e-5
         assert np.max(np.abs(host(M[i]) - Mr[i])) <= 1e-5 * max(1.0, np.max(np.abs(Mr[i])))
         assert np.max(np.abs(got @ got.T - np.eye(rows))) <= 1e-5
+
+
+@pytest.mark.parametrize("n,k", [(256, 64), (300, 100)])
+def test_stiefel_nan_gradient_is_reported(n, k):
+    """A NaN in G reaches every column of the 2k x 2k system, so the elimination meets columns
+    with no finite entry: the step must still pick in-range pivots (row jj, as the textbook
+    algorithm with a NaN-ignoring argmax would), report MUON_ERR_NONFINITE, and leave the
+    device usable for the next call."""
+    Ws = workloads.stiefel_problem(seed=970 + n, batch=2, n=n, k=k)
+    W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+    G = torch.randn(W.shape, device="cuda")
+    G[1, 5, 7] = float("nan")
+    ws = mb.workspace(mb.stiefel_workspace_size(2, n, k))
+    mb.stiefel_cayley_step(W, G, 1e-2, ws)
+    torch.cuda.synchronize()
+    assert mb.device_status(ws) == mb.MUON_ERR_NONFINITE
+    # the same workspace serves a clean step afterwards
+    W2 = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+    G2 = torch.randn(W2.shape, device="cuda")
+    mb.stiefel_cayley_step(W2, G2, 1e-2, ws)
+    assert mb.device_status(ws) == mb.MUON_OK
+    assert orth_err_dev(W2) <= 1e-5

@@ -291,6 +291,25 @@ def test_cayley_preserves_orthonormality_and_woodbury_matches_dense():
         assert np.max(np.abs(Q.T @ Q - np.eye(n))) < 1e-12
 
 
+def test_cayley_doubled_resolvent_form_matches_woodbury():
+    """(I + cA)^-1 (I - cA) = 2 (I + cA)^-1 - I, so with the rank-2k factorisation A = U B the
+    retraction is W - 2 U C^-1 (c B W): the same map as the page's Woodbury steps (b, y = B b,
+    z = C^-1 y, W_new = b - c U z) with y replaced by c B W = [cQ; -cP^T].  Written out here in
+    fp64 from the factorisation and compared with the oracle's Woodbury and dense forms."""
+    r = workloads.rng(43)
+    for (n, k, lr) in [(64, 16, 1e-2), (200, 30, 0.3), (128, 64, 1.0), (96, 96, 2.0)]:
+        W = _orth(r, n, k)
+        V = orc.project_tangent(W, r.standard_normal((n, k)))
+        c = lr / 2
+        P, Q, R = W.T @ V, W.T @ W, V.T @ V
+        C = np.block([[np.eye(k) + c * P, c * Q], [-c * R, np.eye(k) - c * P.T]])
+        z = np.linalg.solve(C, np.concatenate([c * Q, -c * P.T], axis=0))
+        W_new = W - 2 * (V @ z[:k] + W @ z[k:])
+        assert np.max(np.abs(W_new - orc.cayley_woodbury(W, V, lr))) < 1e-12
+        assert np.max(np.abs(W_new - orc.cayley_dense(W, V, lr))) < 1e-12
+        assert orc.orthogonality_error(W_new) < 1e-12
+
+
 def test_cayley_first_order_and_small_lr_limit():
     r = workloads.rng(43)
     n, k = 40, 8
