@@ -233,6 +233,16 @@ __device__ __forceinline__ void cp_async8(double* smem_dst, const double* gmem_s
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// Warp-wide argmax: every lane ends with the largest v and, among lanes holding it, the
+// smallest i (v >= -1, never NaN).
+__device__ __forceinline__ void warp_argmax(double& v, int& i) {
+    double m = v;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+    i = static_cast<int>(__reduce_min_sync(0xffffffffu, v == m ? static_cast<unsigned>(i) : 0x7fffffffu));
+    v = m;
+}
+
 __global__ void __launch_bounds__(1024)
 lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int nb, int* piv, long long piv_stride,
                 unsigned* status) {
@@ -262,23 +272,13 @@ lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int 
             const double v = fabs(colj[r]);
             if (v > best) { best = v; bi = r; }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
-        }
+        warp_argmax(best, bi);   // (largest |a|, then smallest row) over the warp
         if ((tid & 31) == 0) { red_v[tid >> 5] = best; red_i[tid >> 5] = bi; }
         __syncthreads();
         if (tid < 32) {
             best = tid < (nt >> 5) ? red_v[tid] : -1.0;
             bi = tid < (nt >> 5) ? red_i[tid] : jj;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double ov = __shfl_xor_sync(0xffffffffu, best, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
-            }
+            warp_argmax(best, bi);
             if (tid == 0) {
                 s_p = bi;
                 pv[j0 + jj] = j0 + bi;
@@ -294,11 +294,40 @@ lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int 
             cc[p] = t;
         }
         __syncthreads();
+        // rows in pairs (r, r + nt): each pivot-row value is read once for both, and the column
+        // loop runs four columns per trip (the kernel is issue-bound)
         const double piv_v = colj[jj];
-        for (int r = jj + 1 + tid; r < rows; r += nt) {
-            const double l = colj[r] / piv_v;
-            pan[jj * pitch + r] = l;
-            for (int c = jj + 1; c < nb; ++c) pan[c * pitch + r] = fma(-l, pan[c * pitch + jj], pan[c * pitch + r]);
+        for (int r = jj + 1 + tid; r < rows; r += 2 * nt) {
+            const int r1 = r + nt;
+            const bool two = r1 < rows;
+            const double l0 = colj[r] / piv_v;
+            const double l1 = two ? colj[r1] / piv_v : 0.0;
+            pan[jj * pitch + r] = l0;
+            if (two) pan[jj * pitch + r1] = l1;
+            double* p0 = pan + (jj + 1) * pitch + r;
+            const double* u = pan + (jj + 1) * pitch + jj;
+            int c = jj + 1;
+            for (; c + 3 < nb; c += 4, p0 += 4 * pitch, u += 4 * pitch) {
+                const double u0 = u[0], u1 = u[pitch], u2 = u[2 * pitch], u3 = u[3 * pitch];
+                const double a0 = p0[0], a1 = p0[pitch], a2 = p0[2 * pitch], a3 = p0[3 * pitch];
+                p0[0] = fma(-l0, u0, a0);
+                p0[pitch] = fma(-l0, u1, a1);
+                p0[2 * pitch] = fma(-l0, u2, a2);
+                p0[3 * pitch] = fma(-l0, u3, a3);
+                if (two) {
+                    double* q = p0 + nt;
+                    const double b0 = q[0], b1 = q[pitch], b2 = q[2 * pitch], b3 = q[3 * pitch];
+                    q[0] = fma(-l1, u0, b0);
+                    q[pitch] = fma(-l1, u1, b1);
+                    q[2 * pitch] = fma(-l1, u2, b2);
+                    q[3 * pitch] = fma(-l1, u3, b3);
+                }
+            }
+            for (; c < nb; ++c, p0 += pitch, u += pitch) {
+                const double uc = u[0];
+                p0[0] = fma(-l0, uc, p0[0]);
+                if (two) p0[nt] = fma(-l1, uc, p0[nt]);
+            }
         }
         __syncthreads();
     }
