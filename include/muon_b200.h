@@ -141,8 +141,9 @@ MUON_API muon_status muon_step_batched(const muon_matrix_desc* descs, int count,
 
 /* The same step with every G in pinned (page-locked) host memory; W, M and O_out stay on
  * the device.  The set is cut, in descriptor order, into up to MUON_HOST_GRAD_CHUNKS
- * chunks of about equal gradient bytes (the first, whose copy nothing can hide, about half
- * a share).  The chunks' gradients are copied into two staging
+ * chunks whose gradient bytes grow by a factor of 1.5 from one to the next (the first, whose
+ * copy nothing can hide, holds 2% of the bytes for 8 chunks; the staging slots hold the
+ * largest, 35%).  The chunks' gradients are copied into two staging
  * slots of the workspace on a library-owned copy stream, one cudaMemcpyAsync per matrix,
  * while the previous chunk's step runs on `stream`, so the host-to-device transfer
  * overlaps the computation of earlier chunks.  Results equal those of muon_step_batched on

@@ -5,7 +5,7 @@
 // instantiation measured 20% slower than the register-staged fp64 kernel on the LU updates
 // (its 8 x 8 fp64 block leaves too few warps per SM), so only fp32 is launched.  Operand
 // tiles go from global to shared memory by cp.async in 16-byte chunks, zero-filled past the
-// matrix edges, through a 4-deep ring: loads run up to three K-steps ahead of the math and
+// matrix edges, through a 3-deep ring of K-steps of 32: loads run up to two K-steps ahead of the math and
 // need no staging registers.  (The register-staged kernel, profiled on these products,
 // stalled mostly on global-load latency: its prefetch reaches one K-step ahead.)
 #include <cstdint>
@@ -15,13 +15,13 @@
 namespace muon {
 namespace {
 
-constexpr int BM = kSimtBM, BN = kSimtBN, THREADS = kSimtThreads, STAGES = 4;
+constexpr int BM = kSimtBM, BN = kSimtBN, THREADS = kSimtThreads, STAGES = 3;
 static_assert(BM == BN, "square tiles: the A and B tiles share one layout");
 
 template <class Acc>
 struct Cfg {
     static constexpr int V = 16 / static_cast<int>(sizeof(Acc));      // elements per 16-byte chunk
-    static constexpr int BK = sizeof(Acc) == sizeof(float) ? 16 : 8;  // K per stage
+    static constexpr int BK = sizeof(Acc) == sizeof(float) ? 32 : 8;  // K per stage
     static constexpr int PITCH_MN = BM + V;                           // row pitch of [k][mn] tiles
     static constexpr int PITCH_K = BK + V;                            // row pitch of [m][k] tiles
     static constexpr int A_ELEMS = BK * PITCH_MN > BM * PITCH_K ? BK * PITCH_MN : BM * PITCH_K;
