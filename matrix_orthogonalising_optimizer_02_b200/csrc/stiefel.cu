@@ -20,6 +20,8 @@
 #include <algorithm>
 #include <cmath>
 
+#include <cooperative_groups.h>
+
 #include "runtime.cuh"
 #include "simt_async.cuh"
 
@@ -226,6 +228,7 @@ __global__ void block_cast_kernel(const BlockCastItem* __restrict__ items, int c
 // so the per-row sweeps are free of bank conflicts).  Records the pivot row of each column
 // in piv (absolute row indices).
 __host__ __device__ constexpr int panel_pitch(int rows) { return rows | 1; }
+constexpr int kPanelMax = 32;   // widest panel (columns)
 // 8-byte global -> shared copy, zero-filled beyond src_bytes (0 or 8).
 __device__ __forceinline__ void cp_async8(double* smem_dst, const double* gmem_src, int src_bytes) {
     const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
@@ -335,6 +338,129 @@ lu_panel_kernel(double* Aug, long long ld, long long stride, int N, int j0, int 
         const int r = e / nb, c = e % nb;
         a[(j0 + static_cast<long long>(r)) * ld + j0 + c] = pan[c * pitch + r];
     }
+}
+
+// The same panel factorisation spread over a cluster of kPanelCluster CTAs per system: CTA c
+// holds panel rows [c * rp, (c + 1) * rp) in shared memory (column by column, odd pitch),
+// each with its logical row index (a pivot swaps two logical indices; the rows stay where
+// they are, and the write-back puts every row at its logical place).  Per column, one cluster
+// barrier: before it, each CTA writes its candidate (largest |a| over its live rows, smallest
+// logical row on ties) together with that row's nb values into every CTA's shared memory
+// (two buffers, alternating by column); after it, every CTA takes the same pivot, reads the
+// pivot row from its own copy, and eliminates its own live rows.  The pivot choice and the
+// arithmetic per element are those of lu_panel_kernel (l = a / pivot, then a - l u column by
+// column), so results equal it for the same panel width.
+constexpr int kPanelCluster = 8, kPanelClusterThreads = 256;
+__host__ __device__ constexpr int panel_cluster_rows(int rows) { return (rows + kPanelCluster - 1) / kPanelCluster; }
+// Shared memory of lu_panel_cluster_kernel beyond the nb panel columns: the candidate rows,
+// then the rows' logical indices.
+__host__ __device__ constexpr size_t panel_cluster_extra_bytes(int rp) {
+    return static_cast<size_t>(2 * kPanelCluster * kPanelMax) * sizeof(double) + static_cast<size_t>(rp) * sizeof(int);
+}
+__global__ void __launch_bounds__(kPanelClusterThreads)
+lu_panel_cluster_kernel(double* Aug, long long ld, long long stride, int N, int j0, int nb, int* piv,
+                        long long piv_stride, unsigned* status) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ double pan[];   // nb columns of panel_pitch(rp), candidate rows, logical rows
+    constexpr int W = kPanelClusterThreads / 32;
+    __shared__ double red_v[W];
+    __shared__ int red_i[W], red_r[W];
+    __shared__ double cand_v[2][kPanelCluster];
+    __shared__ int cand_i[2][kPanelCluster];
+    __shared__ int s_row;   // this CTA's candidate row (local index)
+    const int me = static_cast<int>(cluster.block_rank());
+    const int sys = static_cast<int>(blockIdx.x) / kPanelCluster;
+    double* a = Aug + sys * stride;
+    int* pv = piv + sys * piv_stride;
+    const int rows = N - j0;
+    const int rp = panel_cluster_rows(rows);
+    const int pitch = panel_pitch(rp);
+    const int r_lo = me * rp;
+    const int nr = max(0, min(rows - r_lo, rp));   // this CTA's rows
+    double* cand_row = pan + static_cast<size_t>(nb) * pitch;             // [2][kPanelCluster][kPanelMax]
+    int* lidx = reinterpret_cast<int*>(cand_row + 2 * kPanelCluster * kPanelMax);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int e = tid; e < nr * nb; e += kPanelClusterThreads) {
+        const int r = e / nb, c = e % nb;
+        cp_async8(pan + c * pitch + r, a + (j0 + static_cast<long long>(r_lo + r)) * ld + j0 + c, 8);
+    }
+    for (int r = tid; r < nr; r += kPanelClusterThreads) lidx[r] = r_lo + r;
+    cp_async_wait_all();
+    __syncthreads();
+    for (int jj = 0; jj < nb; ++jj) {
+        const int buf = jj & 1;
+        const double* colj = pan + jj * pitch;
+        // this CTA's candidate; a NaN ranks as -1, so an all-NaN column pivots on logical row jj
+        double best = -1.0;
+        int bl = 0x7fffffff, br = 0;
+        for (int r = tid; r < nr; r += kPanelClusterThreads) {
+            const int li = lidx[r];
+            if (li < jj) continue;
+            double v = fabs(colj[r]);
+            if (!(v >= 0.0)) v = -1.0;
+            if (v > best || (v == best && li < bl)) { best = v; bl = li; br = r; }
+        }
+        double wv = best;
+        int wl = bl;
+        warp_argmax(wv, wl);
+        const int wr = __shfl_sync(0xffffffffu, br, __ffs(__ballot_sync(0xffffffffu, best == wv && bl == wl)) - 1);
+        if (lane == 0) { red_v[warp] = wv; red_i[warp] = wl; red_r[warp] = wr; }
+        __syncthreads();
+        if (warp == 0) {
+            double v = lane < W ? red_v[lane] : -1.0;
+            int l = lane < W ? red_i[lane] : 0x7fffffff;
+            const double v0 = v;
+            const int l0 = l;
+            warp_argmax(v, l);
+            const int src = __ffs(__ballot_sync(0xffffffffu, v0 == v && l0 == l)) - 1;
+            const int r = __shfl_sync(0xffffffffu, lane < W ? red_r[lane] : 0, src);
+            if (lane == 0) s_row = r;
+            if (lane < kPanelCluster) {   // this CTA's candidate into every CTA's slot `me`
+                *cluster.map_shared_rank(&cand_v[buf][me], lane) = v;
+                *cluster.map_shared_rank(&cand_i[buf][me], lane) = l;
+            }
+        }
+        __syncthreads();
+        {   // the candidate row's values into every CTA's slot `me` (zeros when this CTA has no live row)
+            const int r = s_row;
+            const bool any = nr > 0;
+            for (int e = tid; e < nb * kPanelCluster; e += kPanelClusterThreads) {
+                const int c = e % nb, dst = e / nb;
+                const double val = any ? pan[c * pitch + r] : 0.0;
+                *cluster.map_shared_rank(cand_row + (buf * kPanelCluster + me) * kPanelMax + c, dst) = val;
+            }
+        }
+        cluster.sync();
+        double gv = lane < kPanelCluster ? cand_v[buf][lane] : -1.0;
+        int lp = lane < kPanelCluster ? cand_i[buf][lane] : 0x7fffffff;
+        const double gv0 = gv;
+        const int lp0 = lp;
+        warp_argmax(gv, lp);   // every warp of every CTA reaches the same pivot
+        const int w = __ffs(__ballot_sync(0xffffffffu, gv0 == gv && lp0 == lp)) - 1;   // the CTA holding it
+        const double* prow = cand_row + (buf * kPanelCluster + w) * kPanelMax;
+        if (me == 0 && tid == 0) {
+            pv[j0 + jj] = j0 + lp;
+            if (!(gv > 0.0) || !isfinite(gv)) atomicOr(status, kDevErrNonfinite);
+        }
+        const int pr = (w == me) ? s_row : -1;   // the pivot row here (local index), if any
+        const double piv_v = prow[jj];
+        for (int r = tid; r < nr; r += kPanelClusterThreads) {
+            const int li = lidx[r];
+            if (r == pr) { lidx[r] = jj; continue; }
+            if (li < jj) continue;
+            if (li == jj) lidx[r] = lp;   // the row the pivot displaces takes its logical place
+            const double l = colj[r] / piv_v;
+            pan[jj * pitch + r] = l;
+            for (int c = jj + 1; c < nb; ++c) pan[c * pitch + r] = fma(-l, prow[c], pan[c * pitch + r]);
+        }
+        __syncthreads();
+    }
+    for (int e = tid; e < nr * nb; e += kPanelClusterThreads) {
+        const int r = e / nb, c = e % nb;
+        a[(j0 + static_cast<long long>(lidx[r])) * ld + j0 + c] = pan[c * pitch + r];
+    }
+    cluster.sync();   // no CTA leaves while a peer may still write into its shared memory
 }
 
 // Triangular solves on right-hand columns held in registers.  Each column is shared by G
@@ -482,7 +608,7 @@ __host__ __device__ constexpr size_t swap_ints_bytes(int R, int rows_from_r0) {
 // applied to the block's earlier multiplier columns [c_left, j0) (blocks 0 .. left_blocks - 1)
 // and, with the solve U12 = L11^-1 A12 by the unit-lower nb x nb triangle L11, to the block's
 // columns [j0 + nb, ncols) (the remaining blocks).  nb <= kPanelMax.
-constexpr int kPanelMax = 32, kPanelLanes = 2, kPanelSwapThreads = 128;
+constexpr int kPanelLanes = 2, kPanelSwapThreads = 128;
 constexpr int kPanelSwapCols = kPanelSwapThreads / kPanelLanes;
 constexpr size_t kPanelTriangleBytes = static_cast<size_t>(kPanelMax) * (kPanelMax + 2) * sizeof(double);
 __global__ void __launch_bounds__(kPanelSwapThreads)
@@ -543,6 +669,23 @@ back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, in
 // columns) that fits in kPanelSmem is used.
 constexpr size_t kPanelSmem = 200 * 1024;
 size_t lu_panel_smem(int rows, int nb) { return static_cast<size_t>(panel_pitch(rows)) * nb * sizeof(double); }
+// Shared memory of the cluster panel kernel: this CTA's nb columns of panel_pitch(rows / 8),
+// then the candidate rows and the logical row indices.
+size_t lu_panel_cluster_smem(int rows, int nb) {
+    const int rp = panel_cluster_rows(rows);
+    return static_cast<size_t>(panel_pitch(rp)) * nb * sizeof(double) + panel_cluster_extra_bytes(rp);
+}
+int lu_panel_cluster_width(int rows) {
+    const size_t per_col = static_cast<size_t>(panel_pitch(panel_cluster_rows(rows))) * sizeof(double);
+    const int nb = static_cast<int>((kPanelSmem - panel_cluster_extra_bytes(panel_cluster_rows(rows))) / per_col);
+    return std::max(1, std::min(kPanelMax, nb));
+}
+// Block columns taller than this factorise their panels on a cluster of kPanelCluster CTAs per
+// system (32 columns wide, about 2.8 us per column whatever the height); shorter ones on one
+// CTA per system, whose time per column falls with the height (about 3.6 us at 2048 rows,
+// 1.8 us at 384).  Measured on 16 x 4096 x 1024: 1000 rows 37.44-37.55 ms per step, 1400 37.70,
+// 1800 38.22, 800 37.44, 600 37.51, all on clusters 38.08, none 38.58.
+constexpr int kPanelClusterMinRows = 1000;
 int lu_panel_width(int rows) {
     const int nb = static_cast<int>(kPanelSmem / (static_cast<size_t>(panel_pitch(rows)) * sizeof(double)));
     return std::max(1, std::min(kPanelMax, nb));
@@ -765,13 +908,44 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
     // (K = the width, N = the block's remaining columns) suit the fp64 tensor-core kernel.
     for (int J0 = 0; J0 < N; J0 += kLuBlock) {
         const int JB = std::min(kLuBlock, N - J0);
-        const int widest = std::max(2, lu_panel_width(N - J0) & ~1);
+        const bool on_cluster = N - J0 > kPanelClusterMinRows;
+        const int widest = std::max(2, (on_cluster ? lu_panel_cluster_width(N - J0) : lu_panel_width(N - J0)) & ~1);
         const int npan = (JB + widest - 1) / widest;
         const int nb = std::min(widest, ((JB + npan - 1) / npan + 1) & ~1);
         for (int j0 = J0; j0 < J0 + JB; j0 += nb) {
             const int w = std::min(nb, J0 + JB - j0);
             const size_t smem = lu_panel_smem(N - j0, w);
             const double lu_flops = 2.0 * (N - j0) * w * w * B;
+            if (on_cluster) {
+                const size_t csmem = lu_panel_cluster_smem(N - j0, w);
+                plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
+                    static bool attr_set[64] = {};
+                    int dev = 0;
+                    cudaError_t e = cudaGetDevice(&dev);
+                    if (e != cudaSuccess) return e;
+                    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+                    if (!attr_set[dev]) {
+                        e = cudaFuncSetAttribute(lu_panel_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(kPanelSmem));
+                        if (e != cudaSuccess) return e;
+                        attr_set[dev] = true;
+                    }
+                    cudaLaunchConfig_t cfg = {};
+                    cfg.gridDim = dim3(B * kPanelCluster, 1, 1);
+                    cfg.blockDim = dim3(kPanelClusterThreads, 1, 1);
+                    cfg.dynamicSmemBytes = csmem;
+                    cfg.stream = s;
+                    cudaLaunchAttribute attr;
+                    attr.id = cudaLaunchAttributeClusterDimension;
+                    attr.val.clusterDim.x = kPanelCluster;
+                    attr.val.clusterDim.y = 1;
+                    attr.val.clusterDim.z = 1;
+                    cfg.attrs = &attr;
+                    cfg.numAttrs = 1;
+                    return cudaLaunchKernelEx(&cfg, lu_panel_cluster_kernel, Aug, static_cast<long long>(ld), aug_stride,
+                                              N, j0, w, piv, static_cast<long long>(N), d_status);
+                }});
+            } else
             plan.steps.push_back({MUON_KERNEL_LU, lu_flops, [=](cudaStream_t s) {
                 // the function attribute is per device: set once on each (launches run under
                 // the plan cache's lock)
