@@ -33,7 +33,10 @@ def stiefel_step(W, G, lr):
 
 
 @pytest.mark.parametrize("n,k,lr", [(256, 64, 1e-2), (200, 72, 0.3), (130, 30, 1.0), (64, 16, 1e-2),
-                                     (512, 128, 5e-2), (96, 96, 0.1)])
+                                     (512, 128, 5e-2), (96, 96, 0.1),
+                                     # 2k = 1280: the top block columns (over 1000 rows) factorise their
+                                     # panels on 8-CTA clusters, the lower ones on one CTA per system
+                                     (1536, 640, 1e-2)])
 def test_stiefel_step_matches_oracle(n, k, lr):
     Ws = workloads.stiefel_problem(seed=900 + n, batch=2, n=n, k=k)
     Gs = workloads.stiefel_gradient(900 + n, 0, 2, n, k)
@@ -128,7 +131,7 @@ def test_muon_cayley_wide_batch_matches_transposed_oracle():
         assert np.max(np.abs(got @ got.T - np.eye(rows))) <= 1e-5
 
 
-@pytest.mark.parametrize("n,k", [(256, 64), (300, 100)])
+@pytest.mark.parametrize("n,k", [(256, 64), (300, 100), (1200, 520)])
 def test_stiefel_nan_gradient_is_reported(n, k):
     """A NaN in G reaches every column of the 2k x 2k system, so the elimination meets columns
     with no finite entry: the step must still pick in-range pivots (row jj, as the textbook
