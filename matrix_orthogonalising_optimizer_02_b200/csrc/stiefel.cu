@@ -893,6 +893,36 @@ cudaError_t big_smem(size_t bytes) {
     return cudaSuccess;
 }
 
+// True if lu_panel_cluster_kernel can run on this device with its largest shared memory (one
+// cluster of kPanelCluster CTAs resident); else the plan keeps every panel on one CTA.
+bool panel_clusters_available() {
+    static int state[64] = {};   // 0 unknown, 1 yes, 2 no (plans are built under the cache's lock)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (state[dev] == 0) {
+        bool ok = cudaFuncSetAttribute(lu_panel_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kPanelSmem)) == cudaSuccess;
+        if (ok) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(kPanelCluster, 1, 1);
+            cfg.blockDim = dim3(kPanelClusterThreads, 1, 1);
+            cfg.dynamicSmemBytes = kPanelSmem;
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = kPanelCluster;
+            attr.val.clusterDim.y = 1;
+            attr.val.clusterDim.z = 1;
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            ok = cudaOccupancyMaxActiveClusters(&clusters, lu_panel_cluster_kernel, &cfg) == cudaSuccess && clusters > 0;
+        }
+        cudaGetLastError();   // a refused query leaves no error pending
+        state[dev] = ok ? 1 : 2;
+    }
+    return state[dev] == 1;
+}
+
 // Gaussian elimination with partial pivoting on the augmented fp64 systems [C | y]
 // (N x ncols, row pitch ld, batch B), then back substitution: z overwrites y.
 void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int ncols, int k, int B, long long ld,
@@ -906,9 +936,10 @@ void add_lu_solve(Plan& plan, TableImage& img, double* Aug, int* piv, int N, int
     // shared memory, so the lower block columns take wider panels (fewer, up to kPanelMax
     // columns), split evenly across the block column.  Widths are even, so the in-block updates
     // (K = the width, N = the block's remaining columns) suit the fp64 tensor-core kernel.
+    const bool clusters = panel_clusters_available();
     for (int J0 = 0; J0 < N; J0 += kLuBlock) {
         const int JB = std::min(kLuBlock, N - J0);
-        const bool on_cluster = N - J0 > kPanelClusterMinRows;
+        const bool on_cluster = clusters && N - J0 > kPanelClusterMinRows;
         const int widest = std::max(2, (on_cluster ? lu_panel_cluster_width(N - J0) : lu_panel_width(N - J0)) & ~1);
         const int npan = (JB + widest - 1) / widest;
         const int nb = std::min(widest, ((JB + npan - 1) / npan + 1) & ~1);
