@@ -51,6 +51,22 @@ def test_stiefel_step_matches_oracle(n, k, lr):
         assert orc.orthogonality_error(got[i]) <= 1e-5
 
 
+def test_stiefel_large_k_matches_oracle():
+    """2k = 4096: panels of up to 4096 rows, 512 rows per CTA on the clusters, 22- and 32-column
+    panels, and one-CTA panels below 1000 rows; one step against the oracle."""
+    n, k, lr = 4096, 2048, 1e-2
+    Ws = workloads.stiefel_problem(seed=990, batch=1, n=n, k=k)
+    Gs = workloads.stiefel_gradient(990, 0, 1, n, k)
+    W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+    G = torch.tensor(Gs, dtype=torch.float32, device="cuda")
+    W0 = host(W)
+    stiefel_step(W, G, lr)
+    got = host(W)
+    want = orc.stiefel_cayley_step(W0[0], Gs[0].astype(np.float64), lr)
+    assert np.max(np.abs(got[0] - want)) <= 2e-5
+    assert orc.orthogonality_error(got[0]) <= 1e-5
+
+
 def test_stiefel_zero_lr_is_identity_map():
     Ws = workloads.stiefel_problem(seed=950, batch=1, n=128, k=32)
     W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
