@@ -67,6 +67,24 @@ def test_stiefel_large_k_matches_oracle():
     assert orc.orthogonality_error(got[0]) <= 1e-5
 
 
+def test_stiefel_more_systems_than_one_wave_of_clusters():
+    """24 systems of 1200 x 520 (2k = 1040: the top block column's panels on 8-CTA clusters):
+    192 cluster CTAs, more than the SMs hold at once, so clusters run in waves.  Two sampled
+    systems against the oracle, the manifold invariant on all."""
+    batch, n, k, lr = 24, 1200, 520, 1e-2
+    Ws = workloads.stiefel_problem(seed=991, batch=batch, n=n, k=k)
+    Gs = workloads.stiefel_gradient(991, 0, batch, n, k)
+    W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
+    G = torch.tensor(Gs, dtype=torch.float32, device="cuda")
+    W0 = host(W)
+    stiefel_step(W, G, lr)
+    got = host(W)
+    for i in (0, 17):
+        want = orc.stiefel_cayley_step(W0[i], Gs[i].astype(np.float64), lr)
+        assert np.max(np.abs(got[i] - want)) <= 2e-5
+    assert orth_err_dev(W) <= 1e-5
+
+
 def test_stiefel_zero_lr_is_identity_map():
     Ws = workloads.stiefel_problem(seed=950, batch=1, n=128, k=32)
     W = torch.tensor(Ws, dtype=torch.float32, device="cuda")
