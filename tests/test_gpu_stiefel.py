@@ -36,7 +36,10 @@ def stiefel_step(W, G, lr):
                                      (512, 128, 5e-2), (96, 96, 0.1),
                                      # 2k = 1280: the top block columns (over 1000 rows) factorise their
                                      # panels on 8-CTA clusters, the lower ones on one CTA per system
-                                     (1536, 640, 1e-2)])
+                                     (1536, 640, 1e-2),
+                                     # odd k on the cluster path: no bf16 planes (n % 8 != 0), 3k odd, so
+                                     # the fp64 updates with an odd N fall back to the FMA pipes
+                                     (1100, 515, 1e-2)])
 def test_stiefel_step_matches_oracle(n, k, lr):
     Ws = workloads.stiefel_problem(seed=900 + n, batch=2, n=n, k=k)
     Gs = workloads.stiefel_gradient(900 + n, 0, 2, n, k)
