@@ -139,6 +139,7 @@ struct SplitKItem {
     int M, N, nsplit;
     float alpha, beta;
     int out_f64, e_f64;
+    int vec4;   // four consecutive elements per thread (N % 4 == 0, 16-byte aligned rows)
 };
 __global__ void splitk_reduce_kernel(const SplitKItem* __restrict__ items, int count) {
     const long long b = blockIdx.x;
@@ -149,6 +150,37 @@ __global__ void splitk_reduce_kernel(const SplitKItem* __restrict__ items, int c
     }
     const SplitKItem& it = items[lo];
     const long long mn = static_cast<long long>(it.M) * it.N;
+    if (it.vec4) {   // the same sums, four columns of one row per thread
+        const long long e = ((b - it.block0) * blockDim.x + threadIdx.x) * 4;
+        if (e >= mn) return;
+        double s4[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int j = 0; j < it.nsplit; ++j) {
+            const float4 q = *reinterpret_cast<const float4*>(it.part + j * mn + e);
+            s4[0] += static_cast<double>(q.x); s4[1] += static_cast<double>(q.y);
+            s4[2] += static_cast<double>(q.z); s4[3] += static_cast<double>(q.w);
+        }
+        const long long m = e / it.N, nn = e % it.N;
+        double v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = static_cast<double>(it.alpha) * s4[i];
+        if (it.beta != 0.f) {
+            const long long eo = m * it.ld_e + nn;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                v[i] += static_cast<double>(it.beta) * (it.e_f64 ? static_cast<const double*>(it.E)[eo + i]
+                                                              : static_cast<double>(static_cast<const float*>(it.E)[eo + i]));
+        }
+        const long long oo = m * it.ld_out + nn;
+        if (it.out_f64) {
+            double2* o = reinterpret_cast<double2*>(static_cast<double*>(it.out) + oo);
+            o[0] = make_double2(v[0], v[1]);
+            o[1] = make_double2(v[2], v[3]);
+        } else {
+            *reinterpret_cast<float4*>(static_cast<float*>(it.out) + oo) =
+                make_float4(static_cast<float>(v[0]), static_cast<float>(v[1]), static_cast<float>(v[2]), static_cast<float>(v[3]));
+        }
+        return;
+    }
     const long long e = (b - it.block0) * blockDim.x + threadIdx.x;
     if (e >= mn) return;
     double sum = 0.0;
@@ -174,6 +206,7 @@ struct Split3Item {
     long long block0;
     int rows, cols;
     int src_f64;
+    int vec4;   // four consecutive elements per thread (cols % 4 == 0, aligned rows)
 };
 __global__ void split3_kernel(const Split3Item* __restrict__ items, int count) {
     const long long b = blockIdx.x;
@@ -184,18 +217,53 @@ __global__ void split3_kernel(const Split3Item* __restrict__ items, int count) {
     }
     const Split3Item& it = items[lo];
     const long long n = static_cast<long long>(it.rows) * it.cols;
+    auto split = [](float x, __nv_bfloat16& h, __nv_bfloat16& m, __nv_bfloat16& l) {
+        h = __float2bfloat16_rn(x);
+        const float r1 = x - __bfloat162float(h);
+        m = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(m);
+        l = __float2bfloat16_rn(r2);
+    };
+    if (it.vec4) {   // four columns of one row per thread
+        const long long e = ((b - it.block0) * blockDim.x + threadIdx.x) * 4;
+        if (e >= n) return;
+        const long long r = e / it.cols, c = e % it.cols;
+        float x[4];
+        if (it.src_f64) {
+            const double2* p = reinterpret_cast<const double2*>(static_cast<const double*>(it.src) + r * it.ld + c);
+            const double2 a = p[0], d = p[1];
+            x[0] = static_cast<float>(a.x); x[1] = static_cast<float>(a.y);
+            x[2] = static_cast<float>(d.x); x[3] = static_cast<float>(d.y);
+        } else {
+            const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(it.src) + r * it.ld + c);
+            x[0] = q.x; x[1] = q.y; x[2] = q.z; x[3] = q.w;
+        }
+        __nv_bfloat16 h[4], m[4], l[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split(x[i], h[i], m[i], l[i]);
+        auto put = [&](__nv_bfloat16* dst, const __nv_bfloat16 (&v)[4]) {
+            __nv_bfloat162 p0, p1;
+            p0.x = v[0]; p0.y = v[1]; p1.x = v[2]; p1.y = v[3];
+            uint2 u;
+            u.x = *reinterpret_cast<const uint32_t*>(&p0);
+            u.y = *reinterpret_cast<const uint32_t*>(&p1);
+            *reinterpret_cast<uint2*>(dst + e) = u;
+        };
+        put(it.dst, h);
+        put(it.dst + n, m);
+        put(it.dst + 2 * n, l);
+        return;
+    }
     const long long e = (b - it.block0) * blockDim.x + threadIdx.x;
     if (e >= n) return;
     const long long r = e / it.cols, c = e % it.cols;
     const float x = it.src_f64 ? static_cast<float>(static_cast<const double*>(it.src)[r * it.ld + c])
                                : static_cast<const float*>(it.src)[r * it.ld + c];
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    const float r1 = x - __bfloat162float(h);
-    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(m);
+    __nv_bfloat16 h, m, l;
+    split(x, h, m, l);
     it.dst[e] = h;
     it.dst[n + e] = m;
-    it.dst[2 * n + e] = __float2bfloat16_rn(r2);
+    it.dst[2 * n + e] = l;
 }
 
 // fp32 copy of a k x k block of an fp64 matrix (the same round-to-nearest the SIMT GEMM
@@ -806,6 +874,20 @@ void add_gemm(Plan& plan, TableImage& img, const std::vector<SimtProblem>& all, 
 // The same products with the reduction dimension split into kSplitK chunks: every chunk's
 // fp32 partial goes to `part`, then one launch sums the partials in fp64 and applies
 // alpha, beta and the output type of each original problem.
+// Whether a split-K reduce item / a plane split may take four elements per thread (whole
+// 16-byte vectors on every row), and the blocks of 256 threads it then needs.
+bool splitk_vec4(const SplitKItem& it) {
+    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (it.N % 4 != 0 || !a16(it.part) || !a16(it.out)) return false;
+    return it.out_f64 ? it.ld_out % 2 == 0 : it.ld_out % 4 == 0;
+}
+bool split3_vec4(const Split3Item& it) {
+    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (it.cols % 4 != 0 || (reinterpret_cast<uintptr_t>(it.dst) & 7u) != 0 || !a16(it.src)) return false;
+    return it.src_f64 ? it.ld % 2 == 0 : it.ld % 4 == 0;
+}
+long long elementwise_blocks(long long n, bool vec4) { return vec4 ? (n + 1023) / 1024 : (n + 255) / 256; }
+
 void add_gemm_splitk(Plan& plan, TableImage& img, const std::vector<SimtProblem>& probs, float* part) {
     std::vector<SimtProblem> chunks;
     std::vector<SplitKItem> items;
@@ -835,8 +917,9 @@ void add_gemm_splitk(Plan& plan, TableImage& img, const std::vector<SimtProblem>
         it.part = cur; it.out = P.out; it.E = P.E; it.ld_out = P.ld_out; it.ld_e = P.ld_e;
         it.M = P.M; it.N = P.N; it.nsplit = ns; it.alpha = P.alpha; it.beta = P.beta;
         it.out_f64 = P.out_f64; it.e_f64 = P.e_f64;
+        it.vec4 = splitk_vec4(it) ? 1 : 0;
         it.block0 = block0;
-        block0 += (mn + 255) / 256;
+        block0 += elementwise_blocks(mn, it.vec4 != 0);
         items.push_back(it);
         cur += ns * mn;
     }
@@ -1163,8 +1246,9 @@ void add_tc_splitk(Plan& plan, TableImage& img, const std::vector<TcProblem>& pr
         it.part = cur; it.out = targets[p].out; it.ld_out = targets[p].ld;
         it.M = P.M; it.N = P.N; it.nsplit = ns; it.alpha = targets[p].alpha;
         it.out_f64 = targets[p].out_f64;
+        it.vec4 = splitk_vec4(it) ? 1 : 0;
         it.block0 = block0;
-        block0 += (mn + 255) / 256;
+        block0 += elementwise_blocks(mn, it.vec4 != 0);
         items.push_back(it);
         cur += ns * mn;
     }
@@ -1204,9 +1288,10 @@ void add_split3(Plan& plan, TableImage& img, const std::vector<Split3Item>& in) 
     long long block0 = 0;
     double bytes = 0;
     for (auto& it : items) {
+        it.vec4 = split3_vec4(it) ? 1 : 0;
         it.block0 = block0;
         const long long n = static_cast<long long>(it.rows) * it.cols;
-        block0 += (n + 255) / 256;
+        block0 += elementwise_blocks(n, it.vec4 != 0);
         bytes += n * ((it.src_f64 ? 8.0 : 4.0) + 6.0);
     }
     const Split3Item* di = img.dev<Split3Item>(img.add(items.data(), items.size() * sizeof(Split3Item), kAlign));
