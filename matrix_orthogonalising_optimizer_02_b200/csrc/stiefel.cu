@@ -31,22 +31,33 @@ namespace {
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---------------------------------------------------------------- small kernels
-// S <- (S + S^T) / 2 in place (k x k per matrix).
-__global__ void symmetrize_kernel(float* S, int k, long long stride) {
-    float* s = S + blockIdx.y * stride;
-    const long long total = static_cast<long long>(k) * k;
-    for (long long e = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; e < total;
-         e += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const int i = static_cast<int>(e / k), j = static_cast<int>(e % k);
-        if (j > i) {
-            const float v = 0.5f * (s[static_cast<long long>(i) * k + j] + s[static_cast<long long>(j) * k + i]);
-            s[static_cast<long long>(i) * k + j] = v;
-            s[static_cast<long long>(j) * k + i] = v;
-        }
+// S <- (S + S^T) / 2 in place (k x k per matrix), 32 x 32 tile pairs through shared memory so
+// both the tile and its mirror are read and written along rows.  Block (bj, bi, matrix) with
+// bi <= bj takes tiles (bi, bj) and (bj, bi); the diagonal is left as it is.
+__global__ void __launch_bounds__(256) symmetrize_kernel(float* S, int k, long long stride) {
+    const int bj = blockIdx.x, bi = blockIdx.y;
+    if (bi > bj) return;
+    __shared__ float up[32][33], lo[32][33];
+    float* s = S + blockIdx.z * stride;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
+    for (int r = ty; r < 32; r += 8) {
+        const int i = bi * 32 + r, j = bj * 32 + tx;   // upper tile, row-wise
+        const int i2 = bj * 32 + r, j2 = bi * 32 + tx; // its mirror, row-wise
+        up[r][tx] = (i < k && j < k) ? s[static_cast<long long>(i) * k + j] : 0.f;
+        lo[r][tx] = (i2 < k && j2 < k) ? s[static_cast<long long>(i2) * k + j2] : 0.f;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        // (i, j) in the upper tile with j > i: s[i][j] = s[j][i] = 0.5 (s[i][j] + s[j][i]),
+        // s[j][i] being lo[tx][r]
+        const int i = bi * 32 + r, j = bj * 32 + tx;
+        if (i < k && j < k && j > i) s[static_cast<long long>(i) * k + j] = 0.5f * (up[r][tx] + lo[tx][r]);
+        // mirror row i2 = bj*32 + r, column j2 = bi*32 + tx: the value of (j2, i2) upper pair
+        const int i2 = bj * 32 + r, j2 = bi * 32 + tx;
+        if (i2 < k && j2 < k && i2 > j2) s[static_cast<long long>(i2) * k + j2] = 0.5f * (up[tx][r] + lo[r][tx]);
     }
 }
 
-// D block of the augmented matrix: Aug[k + i][k + j] = -Aug[j][i]   (-c P^T from c P).
 __global__ void aug_neg_transpose_kernel(double* Aug, int k, long long ld, long long stride) {
     double* a = Aug + blockIdx.y * stride;
     const long long total = static_cast<long long>(k) * k;
@@ -275,6 +286,7 @@ struct BlockCastItem {
     long long ld;         // source row pitch
     long long block0;
     int rows, cols;
+    int vec4;             // four consecutive elements per thread (cols % 4 == 0, aligned rows)
 };
 __global__ void block_cast_kernel(const BlockCastItem* __restrict__ items, int count) {
     const long long b = blockIdx.x;
@@ -285,6 +297,16 @@ __global__ void block_cast_kernel(const BlockCastItem* __restrict__ items, int c
     }
     const BlockCastItem& it = items[lo];
     const long long n = static_cast<long long>(it.rows) * it.cols;
+    if (it.vec4) {
+        const long long e = ((b - it.block0) * blockDim.x + threadIdx.x) * 4;
+        if (e >= n) return;
+        const long long r = e / it.cols, c = e % it.cols;
+        const double2* p = reinterpret_cast<const double2*>(it.src + r * it.ld + c);
+        const double2 a = p[0], d = p[1];
+        *reinterpret_cast<float4*>(it.dst + e) =
+            make_float4(static_cast<float>(a.x), static_cast<float>(a.y), static_cast<float>(d.x), static_cast<float>(d.y));
+        return;
+    }
     const long long e = (b - it.block0) * blockDim.x + threadIdx.x;
     if (e >= n) return;
     const long long r = e / it.cols, c = e % it.cols;
@@ -1269,9 +1291,11 @@ void add_block_cast(Plan& plan, TableImage& img, const std::vector<BlockCastItem
     long long block0 = 0;
     double bytes = 0;
     for (auto& it : items) {
+        it.vec4 = (it.cols % 4 == 0 && it.ld % 2 == 0 && (reinterpret_cast<uintptr_t>(it.src) & 15u) == 0 &&
+                   (reinterpret_cast<uintptr_t>(it.dst) & 15u) == 0) ? 1 : 0;
         it.block0 = block0;
         const long long n = static_cast<long long>(it.rows) * it.cols;
-        block0 += (n + 255) / 256;
+        block0 += elementwise_blocks(n, it.vec4 != 0);
         bytes += 12.0 * n;
     }
     const BlockCastItem* di = img.dev<BlockCastItem>(img.add(items.data(), items.size() * sizeof(BlockCastItem), kAlign));
@@ -1370,7 +1394,8 @@ muon_status build_stiefel(Plan& plan, TableImage& img, const StiefelLayout& L, u
         add_gemm_splitk(plan, img, pr, part); pr.clear();
     }
     plan.steps.push_back({MUON_KERNEL_MISC, 8.0 * kk * B, [=](cudaStream_t s) {
-        symmetrize_kernel<<<dim3(std::max(1, std::min<int>(1024, static_cast<int>((kk + 255) / 256))), B), 256, 0, s>>>(S, k, kk);
+        const int tk = (k + 31) / 32;
+        symmetrize_kernel<<<dim3(tk, tk, B), 256, 0, s>>>(S, k, kk);
         return cudaGetLastError();
     }});
     // V = G - W sym(S)
