@@ -715,9 +715,10 @@ lu_swap_trsm_kernel(double* Aug, long long ld, long long stride, int c_left, int
 
 // After a block column J0..J0+JB-1 is factorised: for every column c >= c_lo, apply the
 // block's JB row swaps in order, then solve with the JB x JB unit-lower L11 (U12 = L11^-1 A12).
-// The 128 x 128 triangle (133 KB) is in dynamic shared memory, shared by the block's 64
-// columns (512 threads, 8 lanes per column).
-constexpr int kLuBlock = 128, kLuLanes = 8, kTrsmThreads = 512;
+// The 128 x 128 triangle (133 KB) is in dynamic shared memory, shared by the block's 128
+// columns (512 threads, 4 lanes per column, 32 rows per lane: measured faster than 8 or 16
+// lanes, whose blocks reload the triangle and replay the swaps for fewer columns).
+constexpr int kLuBlock = 128, kLuLanes = 4, kTrsmThreads = 512;
 constexpr size_t kLuTriangleBytes = static_cast<size_t>(kLuBlock) * (kLuBlock + 2) * sizeof(double);
 constexpr int kMaxAugRows = 2 * 4096;   // 2k for the largest k the entry points accept
 __global__ void __launch_bounds__(kTrsmThreads)
@@ -731,9 +732,9 @@ lu_block_swap_trsm_kernel(double* Aug, long long ld, long long stride, int J0, i
 }
 
 // Back substitution on one diagonal block: rows i0..i0+bs-1 of the right-hand columns
-// (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows); 64 columns per block of 512
+// (starting at column rhs0, nrhs of them) <- U_ii^-1 (same rows); 128 columns per block of 512
 // threads, the triangle and the reciprocals of its diagonal in dynamic shared memory.
-constexpr int kBackBlock = 128, kBackLanes = 8, kBackPitch = kBackBlock + 2;
+constexpr int kBackBlock = 128, kBackLanes = 4, kBackPitch = kBackBlock + 2;
 constexpr size_t kBackSmemBytes = (static_cast<size_t>(kBackBlock) * kBackPitch + kBackBlock) * sizeof(double);
 __global__ void __launch_bounds__(kTrsmThreads)
 back_diag_kernel(double* Aug, long long ld, long long stride, int i0, int bs, int rhs0, int nrhs) {
