@@ -6,8 +6,10 @@
 //
 // 256 threads = 8 warps in a 2 (M) x 4 (N) grid, each warp 64 x 32 = 4 x 4 tiles of 16 x 8.
 // Operand tiles go global -> shared by cp.async in 16-byte chunks (zero-filled outside the
-// matrices) through a 3-stage ring of K-steps of 16.  The first stages of a CTA's next tile
-// are issued before the epilogue of the current one, so their latency hides behind it, and
+// matrices) through a 2-stage ring of K-steps of 16 (measured faster than 3 or 4 stages,
+// likely because the smaller shared-memory footprint leaves more L1 to the epilogue).  The
+// first K-step of a CTA's next tile is issued before the epilogue of the current one, so its
+// latency hides behind it, and
 // the epilogue reads a half tile of E before it stores any result: E may be the output itself,
 // so loads placed after stores would each wait out a full memory latency (the LU's K = 128
 // updates spend about as long in the epilogue as in the MMAs).  Shared pitches are chosen so
@@ -21,7 +23,7 @@
 namespace muon {
 namespace {
 
-constexpr int BM = 128, BN = 128, BKD = 16, STAGES = 3, THREADS = 256;
+constexpr int BM = 128, BN = 128, BKD = 16, STAGES = 2, THREADS = 256;
 constexpr int PA = BKD + 4;     // doubles per A row ([m][k])
 constexpr int PB = BN + 4;      // doubles per B row ([k][n])
 constexpr int A_ELEMS = BM * PA, B_ELEMS = BKD * PB;
