@@ -5,9 +5,10 @@
 // instantiation measured 20% slower than the register-staged fp64 kernel on the LU updates
 // (its 8 x 8 fp64 block leaves too few warps per SM), so only fp32 is launched.  Operand
 // tiles go from global to shared memory by cp.async in 16-byte chunks, zero-filled past the
-// matrix edges, through a 3-deep ring of K-steps of 32: loads run up to two K-steps ahead of the math and
-// need no staging registers.  (The register-staged kernel, profiled on these products,
-// stalled mostly on global-load latency: its prefetch reaches one K-step ahead.)
+// matrix edges, through a 2-deep ring of K-steps of 32 (measured faster than 3 or 4 stages):
+// the next K-step loads while the current one computes, with no staging registers.  (The
+// register-staged kernel, profiled on these products, stalled mostly on global-load latency:
+// its loads pass through registers.)
 #include <cstdint>
 
 #include "simt_async.cuh"
@@ -15,7 +16,7 @@
 namespace muon {
 namespace {
 
-constexpr int BM = kSimtBM, BN = kSimtBN, THREADS = kSimtThreads, STAGES = 3;
+constexpr int BM = kSimtBM, BN = kSimtBN, THREADS = kSimtThreads, STAGES = 2;
 static_assert(BM == BN, "square tiles: the A and B tiles share one layout");
 
 template <class Acc>

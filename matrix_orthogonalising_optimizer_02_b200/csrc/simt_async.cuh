@@ -15,7 +15,7 @@ namespace muon {
 bool simt_async_suits(const std::vector<SimtProblem>& probs, bool* a_kc);
 
 // Same contract and tile codes as simt_gemm_launch with fp32 accumulation (128 x 128 tiles),
-// operand tiles staged by cp.async through a 3-deep shared-memory ring of K-steps of 32.
+// operand tiles staged by cp.async through a 2-deep shared-memory ring of K-steps of 32.
 cudaError_t simt_gemm_async_launch(const SimtProblem* d_probs, const uint32_t* d_tiles, int num_tiles,
                                    cudaStream_t stream, bool a_kc);
 
