@@ -80,10 +80,6 @@ __device__ __forceinline__ void store_tile(Acc (*s)[BM + PAD], bool k_contig, in
     }
 }
 
-__device__ __forceinline__ void load4(const float* p, float (&v)[4], int o) {
-    const float4 q = *reinterpret_cast<const float4*>(p);
-    v[o] = q.x; v[o + 1] = q.y; v[o + 2] = q.z; v[o + 3] = q.w;
-}
 __device__ __forceinline__ void load4(const double* p, double (&v)[8], int o) {
     const double2 a = *reinterpret_cast<const double2*>(p);
     const double2 b = *reinterpret_cast<const double2*>(p + 2);
