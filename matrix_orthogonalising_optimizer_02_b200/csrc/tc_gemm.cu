@@ -79,6 +79,27 @@ __device__ __forceinline__ void cp_async_wait_group() {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// Transpose one 32 x 32 bf16 chunk held in staging layout (row r, 16-byte segment s at
+// stg_off64(r, s)) into `dst` in the same layout: dst row c, column r = src row r, column c.
+// Per column strip j, ldmatrix.trans reads the four 8 x 8 blocks (rows 8i.., segment j) of
+// the strip and hands each lane its pieces of their transposes; stmatrix writes them as the
+// blocks (rows 8j.., segment i) of dst.  Lane L addresses row L of src (ldmatrix: lanes
+// 8i..8i+7 give block i's rows) and row 8j + (L & 7), segment L >> 3 of dst.  Both sides hit
+// each bank group once per 8 rows.
+__device__ __forceinline__ void stg_transpose32(const uint8_t* src, uint8_t* dst, int lane) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t r0, r1, r2, r3;
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                     : "r"(smem_u32(src + stg_off64(lane, j)))
+                     : "memory");
+        asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};"
+                     ::"r"(smem_u32(dst + stg_off64(8 * j + (lane & 7), lane >> 3))), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                     : "memory");
+    }
+}
+
 __device__ __forceinline__ void store_bf16x8(__nv_bfloat16* dst, const float* v) {
     uint4 w;
     w.x = pack_bf16x2(v[0], v[1]);
@@ -476,22 +497,11 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                                 if (rr < P.M && cc < P.N)
                                     *reinterpret_cast<uint4*>(o + static_cast<size_t>(rr) * P.ld + cc) = val;
                             }
-                            __syncwarp();
-                        }
-                        if (sym) {
-                            // mirror: lane L writes column L of the transposed chunk, which then
-                            // leaves as 8 rows x 64 B per instruction
-#pragma unroll 1
-                            for (int pl = 0; pl < (lo_out ? 2 : 1); ++pl) {
-#pragma unroll
-                                for (int j = 0; j < 32; ++j) {
-                                    const __nv_bfloat16 hv = __float2bfloat16_rn(v[j]);
-                                    const __nv_bfloat16 bv =
-                                        pl == 0 ? hv : __float2bfloat16_rn(v[j] - __bfloat162float(hv));
-                                    *reinterpret_cast<__nv_bfloat16*>(stg_t + stg_off64(j, lane >> 3) + 2 * (lane & 7)) = bv;
-                                }
+                            if (sym) {
+                                // mirror: the staged plane transposed into stg_t, which then
+                                // leaves as 8 rows x 64 B per instruction
+                                stg_transpose32(stg, stg_t, lane);
                                 __syncwarp();
-                                __nv_bfloat16* o = static_cast<__nv_bfloat16*>(P.out[pl]);
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
                                     const int rr = col0 + crow + 8 * i;     // mirrored row
@@ -500,8 +510,8 @@ tc_gemm_kernel(const TcProblem* __restrict__ probs, const uint32_t* __restrict__
                                     if (rr < P.N && cc < P.M)
                                         *reinterpret_cast<uint4*>(o + static_cast<size_t>(rr) * P.ld + cc) = val;
                                 }
-                                __syncwarp();
                             }
+                            __syncwarp();
                         }
                     }
                 }
